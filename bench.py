@@ -1,0 +1,373 @@
+#!/usr/bin/env python
+"""Benchmark: BCJR forward+backward over the S = 2^16, k = 2 bitshift trellis.
+
+Workload: a 2048 x 8192 projection matrix of iid N(0,1) weights (stand-in for
+Hadamard-incoherent LLM weights) split into 65536 sequences of 256 steps,
+65536 iid N(0,1) codewords, one annealing sweep with T geometric from 0.3 to
+0.005 (8 temperatures).  One step = one forward call (soft codeword) and one
+backward call (dL/dw, dL/dcodebook) at the next temperature of the sweep,
+through the library's C ABI, with the upstream gradient iid N(0,1).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line on rank 0.  Under torchrun each rank holds its own
+projection matrix (weak scaling) with a shared codebook whose gradient is
+summed over ranks by one NCCL all-reduce per step.
+
+`--impl reference` times the float64 CPU oracle on the host cores instead, on
+a bounded sample of the same workload (whole sequences), same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import bcjr_inputs as I  # noqa: E402
+
+METRIC = "BCJR fwd+bwd weights/s and state-updates/s at S=2^16,k=2; % of exp-pipe peak"
+WORKLOAD = "proj2048x8192_L16_k2"
+MUFU_OPS_PER_CLK_PER_SM = 16      # ex2/lg2 throughput per SM per clock (compute capability 10.0)
+ALG_MUFU_PER_STATE_STEP = 4       # one forward and one backward log-sum-exp in each of the two calls
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=8)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--checkpoint-interval", type=int, default=1)
+    ap.add_argument("--n-seq", type=int, default=0,
+                    help="sequences per GPU (default: the workload's 65536); smaller only for profiling")
+    return ap.parse_args()
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region
+# --------------------------------------------------------------------------
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------
+# CPU oracle (reported baseline, and the --impl reference arm)
+# --------------------------------------------------------------------------
+def oracle_sample_rate(n_seq_sample: int, temps):
+    """Time the float64 oracle, fwd+bwd, on the first sequences of the workload."""
+    import oracle
+    W = I.WORKLOADS[WORKLOAD]
+    L, k, n = W["state_bits"], W["k"], W["seq_len"]
+    c = I.codebook(1 << L)
+    w = I.weights(n_seq_sample, n)
+    g = I.upstream_grad(n_seq_sample, n)
+    cores = len(os.sched_getaffinity(0))
+    threads = min(cores, n_seq_sample)
+    t0 = time.perf_counter()
+    for T in temps:
+        oracle.forward(w, c, T, L, k, nthreads=threads)
+        oracle.backward(g, w, c, T, L, k, nthreads=threads)
+    dt = time.perf_counter() - t0
+    weights = n_seq_sample * n * len(temps)
+    return weights / dt, threads, dt
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    W = I.WORKLOADS[WORKLOAD]
+    L, n = W["state_bits"], W["seq_len"]
+    temps = W["T"]
+    cores = len(os.sched_getaffinity(0))
+    sample = max(1, min(cores, 16))
+    import oracle
+    oracle.build()
+    times = []
+    for i in range(args.warmup + args.steps):
+        rate, threads, dt = oracle_sample_rate(sample, [temps[i % len(temps)]])
+        if i >= args.warmup:
+            times.append(dt)
+    ms = 1e3 * statistics.mean(times)
+    value = sample * n / (ms / 1e3)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "weights/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "state_updates_per_s": value * (1 << L),
+        "config": _config(args.gpus, args.checkpoint_interval),
+        "cpu_baseline": {"value": value, "unit": "weights/s", "cores": min(cores, sample), "kind": "oracle",
+                         "sample": f"{sample} whole sequences of the workload per step (fwd+bwd, float64, "
+                                   f"OpenMP over sequences), T cycling through the sweep"},
+        "e2e": {"value": value, "unit": "weights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(n_gpus, C, n_seq=None):
+    W = I.WORKLOADS[WORKLOAD]
+    n_seq = n_seq or W["n_seq"]
+    return {"workload": WORKLOAD if n_seq == W["n_seq"] else f"{WORKLOAD}[first {n_seq} rows]",
+            "state_bits": W["state_bits"], "k": W["k"], "seq_len": W["seq_len"],
+            "n_seq_per_gpu": n_seq, "weights_per_gpu": n_seq * W["seq_len"],
+            "T_schedule": [round(t, 6) for t in W["T"]], "checkpoint_interval": C,
+            "parallelism": f"dp{n_gpus}",
+            "l2": "no flush: each step streams > 1 GiB of workspace and 256 MiB of inputs/outputs, "
+                  "both larger than the 126 MB L2"}
+
+
+# --------------------------------------------------------------------------
+# GPU arm
+# --------------------------------------------------------------------------
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        return json.load(open(p))
+    except Exception:
+        return {}
+
+
+def load_traffic():
+    """dram bytes per launch of the dominant kernel from the committed ncu summary, if current."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        return json.load(open(p))
+    except Exception:
+        return {}
+
+
+def run_gpu(args):
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    import differentiable_bcjr_b200 as B
+
+    W = I.WORKLOADS[WORKLOAD]
+    L, k, n, N, temps = W["state_bits"], W["k"], W["seq_len"], W["n_seq"], W["T"]
+    if args.n_seq > 0:
+        N = args.n_seq
+    S = 1 << L
+    C = args.checkpoint_interval
+    # each rank: its own projection matrix (seed offset by rank), shared codebook
+    c_h = I.codebook(S)
+    w_h = I.weights(N, n, seed=I.SEED_WEIGHTS + 100 * rank)
+    g_h = I.upstream_grad(N, n, seed=I.SEED_UPSTREAM + 100 * rank)
+    c = c_h.to(dev)
+    w = w_h.to(dev)
+    g = g_h.to(dev)
+    w_hat = torch.empty_like(w)
+    grad_c = torch.zeros(S, device=dev)
+    ws_f = B.Workspace(dev)
+    ws_b = B.Workspace(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i, w_in, g_in, what_out):
+        T = temps[i % len(temps)]
+        B.bcjr_forward(w_in, c, T, L, k, checkpoint_interval=C, ws=ws_f, out=what_out)
+        gw, gc = B.bcjr_backward(g_in, w_in, c, what_out, T, L, k, checkpoint_interval=C, ws=ws_b,
+                                 grad_codebook=grad_c, accumulate_codebook=False)
+        if world > 1:
+            torch.distributed.all_reduce(gc)
+        return gw, gc
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+
+    for i in range(args.warmup):
+        step(i, w, g, w_hat)
+    barrier()
+
+    # ---- device-timed region: inputs resident in HBM ----
+    sampler = ClockSampler(local)
+    sampler.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    start.record(stream)
+    for i in range(args.steps):
+        T = temps[i % len(temps)]
+        ev[i][0].record(stream)
+        B.bcjr_forward(w, c, T, L, k, checkpoint_interval=C, ws=ws_f, out=w_hat)
+        ev[i][1].record(stream)
+        gw, gc = B.bcjr_backward(g, w, c, w_hat, T, L, k, checkpoint_interval=C, ws=ws_b,
+                                 grad_codebook=grad_c, accumulate_codebook=False)
+        ev[i][2].record(stream)
+        if world > 1:
+            torch.distributed.all_reduce(gc)
+    end.record(stream)
+    barrier()
+    clocks = sampler.stop()
+    elapsed_ms = start.elapsed_time(end)
+    fwd_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    bwd_ms = [b.elapsed_time(cc) for _, b, cc in ev]
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / args.steps
+    weights_total = world * N * n
+    value = weights_total / (ms_per_step / 1e3)
+
+    # ---- end-to-end through the public API with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        w_pin = w_h.pin_memory()
+        g_pin = g_h.pin_memory()
+        what_pin = torch.empty_like(w_h).pin_memory()
+        gw_pin = torch.empty_like(w_h).pin_memory()
+        gc_pin = torch.empty(S).pin_memory()
+        w_d = torch.empty_like(w)
+        g_d = torch.empty_like(g)
+        h2d = w_pin.numel() * 4 + g_pin.numel() * 4
+        d2h = what_pin.numel() * 4 + gw_pin.numel() * 4 + gc_pin.numel() * 4
+        barrier()
+        s2 = torch.cuda.Event(enable_timing=True)
+        e2 = torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for i in range(args.steps):
+            w_d.copy_(w_pin, non_blocking=True)
+            g_d.copy_(g_pin, non_blocking=True)
+            gw, gc = step(i, w_d, g_d, w_hat)
+            what_pin.copy_(w_hat, non_blocking=True)
+            gw_pin.copy_(gw, non_blocking=True)
+            gc_pin.copy_(gc, non_blocking=True)
+        e2.record(stream)
+        barrier()
+        e2e_ms = s2.elapsed_time(e2)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": weights_total / (e2e_ms / args.steps / 1e3), "unit": "weights/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps}
+
+    if rank == 0:
+        peaks = load_peaks()
+        props = torch.cuda.get_device_properties(dev)
+        sms = props.multi_processor_count
+        max_mhz = float(peaks.get("sm_max_mhz", 1965.0))
+        mufu_peak = MUFU_OPS_PER_CLK_PER_SM * sms * max_mhz * 1e6          # ops/s at the max clock
+        state_steps = N * n * S
+        # dominant kernel: the backward launch (2 log-sum-exp sweeps per state-step)
+        bwd_avg_s = statistics.mean(bwd_ms) / 1e3
+        fwd_avg_s = statistics.mean(fwd_ms) / 1e3
+        achieved = 2 * state_steps / bwd_avg_s
+        traffic = load_traffic().get("bwd_dram_bytes_per_launch")
+        frac_total = ALG_MUFU_PER_STATE_STEP * state_steps * world / (ms_per_step / 1e3) / (mufu_peak * world)
+        line = {
+            "metric": METRIC, "value": value, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": _config(world, C, N),
+            "state_updates_per_s": value * S,
+            "exp_roofline_frac": frac_total,
+            "roofline": {"bound": "alu", "pipe": "MUFU (ex2/lg2)", "achieved": achieved / 1e12,
+                         "peak": mufu_peak / 1e12, "unit": "Texp/s", "frac": achieved / mufu_peak,
+                         "traffic": traffic, "kernel": "fb_kernel<adjoint> (bcjr_backward)",
+                         "peak_source": f"{MUFU_OPS_PER_CLK_PER_SM} ops/clk/SM x {sms} SMs x {max_mhz:.0f} MHz "
+                                        "(sm_max_mhz of MEASURED_PEAKS.json)"},
+            "kernels_ms": {"bcjr_forward": 1e3 * fwd_avg_s, "bcjr_backward": 1e3 * bwd_avg_s},
+            "gpu_launches": 3 * args.steps,
+            "clocks": clocks,
+        }
+        if e2e is not None:
+            line["e2e"] = e2e
+        if world == 1 and not args.no_cpu_baseline:
+            try:
+                cores = len(os.sched_getaffinity(0))
+                sample = max(1, min(cores, 16))
+                rate, threads, dt = oracle_sample_rate(sample, [temps[0]])
+                line["cpu_baseline"] = {"value": rate, "unit": "weights/s", "cores": threads, "kind": "oracle",
+                                        "sample": f"{sample} whole sequences (fwd+bwd at T={temps[0]}), "
+                                                  f"{dt:.1f} s of CPU work"}
+            except Exception as e:  # pragma: no cover
+                line["cpu_baseline"] = {"value": None, "error": str(e)}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,269 @@
+"""differentiable_bcjr_b200 -- B200 (sm_100a) kernels for the BCJR-QAT hot path.
+
+A thin ctypes binding over libbcjr.so (C ABI in include/bcjr.h).  This module
+only marshals arguments: PyTorch supplies device memory and the current CUDA
+stream, every step of the computation runs in the library's kernels.  There
+is no CPU fallback: if the library is missing or no CUDA device is present,
+the calls raise.
+
+  bcjr_forward(w, codebook, T, state_bits, k)        -> (w_hat, marginals|None, log_z)
+  bcjr_backward(grad_w_hat, w, codebook, w_hat, T, state_bits, k) -> (grad_w, grad_codebook)
+  viterbi_decode(w, codebook, state_bits, k)          -> (states, w_hard)
+  bcjr_dense_forward / bcjr_dense_backward            (fully connected trellis)
+  SoftTrellisQuant                                    torch.autograd.Function
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "LIB_PATH", "lib", "BCJRError", "bcjr_forward", "bcjr_backward", "viterbi_decode",
+    "bcjr_dense_forward", "bcjr_dense_backward", "workspace_size", "Workspace",
+    "SoftTrellisQuant", "soft_quantize", "OP_FORWARD", "OP_BACKWARD", "OP_VITERBI",
+    "OP_DENSE_FORWARD", "OP_DENSE_BACKWARD", "STATUS",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbcjr.so")
+
+OP_FORWARD, OP_BACKWARD, OP_VITERBI, OP_DENSE_FORWARD, OP_DENSE_BACKWARD = range(5)
+STATUS = {0: "BCJR_OK", 1: "BCJR_ERR_INVALID_ARG", 2: "BCJR_ERR_UNSUPPORTED", 3: "BCJR_ERR_WORKSPACE",
+          4: "BCJR_ERR_CUDA", 5: "BCJR_ERR_TIMEOUT", 6: "BCJR_ERR_NONFINITE"}
+
+
+class BCJRError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {lib().bcjr_status_string(status).decode()}")
+
+
+class Options(ctypes.Structure):
+    _fields_ = [("checkpoint_interval", ctypes.c_int), ("reserved", ctypes.c_int * 7)]
+
+
+_lib = None
+_P = ctypes.c_void_p
+_F = ctypes.c_float
+_I = ctypes.c_int
+_Z = ctypes.c_size_t
+
+_SIGS = {
+    "bcjr_workspace_size": (_Z, [_I, _I, _I, _I, _I, ctypes.POINTER(Options)]),
+    "bcjr_forward": (_I, [_P, _P, _F, _I, _I, _I, _I, _P, _P, _P, ctypes.POINTER(Options), _P, _Z, _P]),
+    "bcjr_backward": (_I, [_P, _P, _P, _P, _F, _I, _I, _I, _I, _P, _P, _I, ctypes.POINTER(Options), _P, _Z,
+                           _P]),
+    "viterbi_decode": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _Z, _P]),
+    "bcjr_dense_forward": (_I, [_P, _P, _P, _F, _I, _I, _I, _P, _P, _P, ctypes.POINTER(Options), _P, _Z, _P]),
+    "bcjr_dense_backward": (_I, [_P, _P, _P, _P, _P, _F, _I, _I, _I, _P, _P, _I, ctypes.POINTER(Options), _P,
+                                 _Z, _P]),
+    "bcjr_get_status": (_I, [_P, _P]),
+    "bcjr_status_string": (ctypes.c_char_p, [_I]),
+    "bcjr_version": (_I, []),
+}
+
+
+def lib():
+    """The loaded libbcjr (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m differentiable_bcjr_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _opts(checkpoint_interval: int = 0):
+    o = Options()
+    o.checkpoint_interval = int(checkpoint_interval)
+    return o
+
+
+def _stream(device=None) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("libbcjr works on CUDA tensors only (no CPU path)")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def workspace_size(op: int, state_bits: int, k: int, seq_len: int, n_seq: int, checkpoint_interval: int = 0) -> int:
+    o = _opts(checkpoint_interval)
+    return int(lib().bcjr_workspace_size(op, state_bits, k, seq_len, n_seq, ctypes.byref(o)))
+
+
+class Workspace:
+    """A reusable device workspace that grows on demand (one per stream)."""
+
+    def __init__(self, device=None):
+        self.device = torch.device(device or "cuda")
+        self.buf = None
+
+    def get(self, nbytes: int) -> torch.Tensor:
+        nbytes = max(int(nbytes), 256)
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        return self.buf
+
+
+_default_ws = {}
+
+
+def _ws(device, nbytes, ws):
+    if ws is None:
+        key = (torch.device(device).index, torch.cuda.current_stream(device).cuda_stream)
+        ws = _default_ws.setdefault(key, Workspace(device))
+    return ws.get(nbytes)
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise BCJRError(status, what)
+
+
+def get_status(ws_tensor: torch.Tensor) -> int:
+    return int(lib().bcjr_get_status(ws_tensor.data_ptr(), _stream(ws_tensor.device)))
+
+
+def bcjr_forward(w, codebook, T, state_bits, k, want_marginals=False, checkpoint_interval=0, ws=None,
+                 out=None):
+    """Soft codeword of every row of w [N][n] (float32, CUDA).  Returns
+    (w_hat [N][n], marginals [N][n][S] or None, log_z [N])."""
+    _need_cuda(w, codebook)
+    N, n = w.shape
+    S = 1 << state_bits
+    dev = w.device
+    w_hat = out if out is not None else torch.empty((N, n), dtype=torch.float32, device=dev)
+    marg = torch.empty((N, n, S), dtype=torch.float32, device=dev) if want_marginals else None
+    log_z = torch.empty((N,), dtype=torch.float32, device=dev)
+    o = _opts(checkpoint_interval)
+    nbytes = lib().bcjr_workspace_size(OP_FORWARD, state_bits, k, n, N, ctypes.byref(o))
+    if nbytes == 0:
+        raise BCJRError(2, "bcjr_workspace_size")
+    wsb = _ws(dev, nbytes, ws)
+    _check(lib().bcjr_forward(_ptr(w), _ptr(codebook), float(T), state_bits, k, n, N, _ptr(w_hat), _ptr(marg),
+                              _ptr(log_z), ctypes.byref(o), _ptr(wsb), wsb.numel(), _stream(dev)),
+           "bcjr_forward")
+    return w_hat, marg, log_z
+
+
+def bcjr_backward(grad_w_hat, w, codebook, w_hat, T, state_bits, k, checkpoint_interval=0, ws=None,
+                  grad_codebook=None, accumulate_codebook=False):
+    """VJP of the soft codeword.  Returns (grad_w [N][n], grad_codebook [S])."""
+    _need_cuda(grad_w_hat, w, codebook, w_hat)
+    N, n = w.shape
+    S = 1 << state_bits
+    dev = w.device
+    grad_w = torch.empty((N, n), dtype=torch.float32, device=dev)
+    if grad_codebook is None:
+        grad_codebook = torch.empty((S,), dtype=torch.float32, device=dev)
+        accumulate_codebook = False
+    o = _opts(checkpoint_interval)
+    nbytes = lib().bcjr_workspace_size(OP_BACKWARD, state_bits, k, n, N, ctypes.byref(o))
+    if nbytes == 0:
+        raise BCJRError(2, "bcjr_workspace_size")
+    wsb = _ws(dev, nbytes, ws)
+    _check(lib().bcjr_backward(_ptr(grad_w_hat), _ptr(w), _ptr(codebook), _ptr(w_hat), float(T), state_bits, k,
+                               n, N, _ptr(grad_w), _ptr(grad_codebook), int(bool(accumulate_codebook)),
+                               ctypes.byref(o), _ptr(wsb), wsb.numel(), _stream(dev)), "bcjr_backward")
+    return grad_w, grad_codebook
+
+
+def viterbi_decode(w, codebook, state_bits, k, ws=None):
+    """Hard (T -> 0) decode.  Returns (states int32 [N][n], w_hard [N][n])."""
+    _need_cuda(w, codebook)
+    N, n = w.shape
+    dev = w.device
+    states = torch.empty((N, n), dtype=torch.int32, device=dev)
+    w_hard = torch.empty((N, n), dtype=torch.float32, device=dev)
+    nbytes = lib().bcjr_workspace_size(OP_VITERBI, state_bits, k, n, N, None)
+    if nbytes == 0:
+        raise BCJRError(2, "bcjr_workspace_size")
+    wsb = _ws(dev, nbytes, ws)
+    _check(lib().viterbi_decode(_ptr(w), _ptr(codebook), state_bits, k, n, N, _ptr(states), _ptr(w_hard),
+                                _ptr(wsb), wsb.numel(), _stream(dev)), "viterbi_decode")
+    return states, w_hard
+
+
+def _log2_states(S: int) -> int:
+    b = S.bit_length() - 1
+    if 1 << b != S:
+        raise ValueError("n_states must be a power of two")
+    return b
+
+
+def bcjr_dense_forward(w, codebook, log_trans, T, want_marginals=False, checkpoint_interval=0, ws=None):
+    _need_cuda(w, codebook, log_trans)
+    N, n = w.shape
+    S = codebook.shape[0]
+    dev = w.device
+    w_hat = torch.empty((N, n), dtype=torch.float32, device=dev)
+    marg = torch.empty((N, n, S), dtype=torch.float32, device=dev) if want_marginals else None
+    log_z = torch.empty((N,), dtype=torch.float32, device=dev)
+    o = _opts(checkpoint_interval)
+    nbytes = lib().bcjr_workspace_size(OP_DENSE_FORWARD, _log2_states(S), 0, n, N, ctypes.byref(o))
+    if nbytes == 0:
+        raise BCJRError(2, "bcjr_workspace_size")
+    wsb = _ws(dev, nbytes, ws)
+    _check(lib().bcjr_dense_forward(_ptr(w), _ptr(codebook), _ptr(log_trans), float(T), S, n, N, _ptr(w_hat),
+                                    _ptr(marg), _ptr(log_z), ctypes.byref(o), _ptr(wsb), wsb.numel(),
+                                    _stream(dev)), "bcjr_dense_forward")
+    return w_hat, marg, log_z
+
+
+def bcjr_dense_backward(grad_w_hat, w, codebook, log_trans, w_hat, T, checkpoint_interval=0, ws=None):
+    _need_cuda(grad_w_hat, w, codebook, log_trans, w_hat)
+    N, n = w.shape
+    S = codebook.shape[0]
+    dev = w.device
+    grad_w = torch.empty((N, n), dtype=torch.float32, device=dev)
+    grad_c = torch.empty((S,), dtype=torch.float32, device=dev)
+    o = _opts(checkpoint_interval)
+    nbytes = lib().bcjr_workspace_size(OP_DENSE_BACKWARD, _log2_states(S), 0, n, N, ctypes.byref(o))
+    if nbytes == 0:
+        raise BCJRError(2, "bcjr_workspace_size")
+    wsb = _ws(dev, nbytes, ws)
+    _check(lib().bcjr_dense_backward(_ptr(grad_w_hat), _ptr(w), _ptr(codebook), _ptr(log_trans), _ptr(w_hat),
+                                     float(T), S, n, N, _ptr(grad_w), _ptr(grad_c), 0, ctypes.byref(o), _ptr(wsb),
+                                     wsb.numel(), _stream(dev)), "bcjr_dense_backward")
+    return grad_w, grad_c
+
+
+class SoftTrellisQuant(torch.autograd.Function):
+    """w_hat = BCJR soft codeword of w at temperature T (differentiable in w and codebook)."""
+
+    @staticmethod
+    def forward(ctx, w, codebook, T, state_bits, k):
+        w_c = w.contiguous()
+        c_c = codebook.contiguous()
+        w_hat, _, _ = bcjr_forward(w_c, c_c, T, state_bits, k)
+        ctx.save_for_backward(w_c, c_c, w_hat)
+        ctx.cfg = (float(T), int(state_bits), int(k))
+        return w_hat
+
+    @staticmethod
+    def backward(ctx, grad_w_hat):
+        w, c, w_hat = ctx.saved_tensors
+        T, L, k = ctx.cfg
+        gw, gc = bcjr_backward(grad_w_hat.contiguous().float(), w, c, w_hat, T, L, k)
+        return gw, gc, None, None, None
+
+
+def soft_quantize(w, codebook, T, state_bits, k):
+    return SoftTrellisQuant.apply(w, codebook, T, state_bits, k)

@@ -1,0 +1,147 @@
+// bcjr_device.cuh -- device-side building blocks of the bitshift-trellis kernels.
+//
+// Team geometry.  One weight sequence is processed by a "team" of S/16
+// threads; every thread owns the same 16 trellis states for the whole launch,
+// so its 16 codewords stay in registers and its 16 codebook-gradient
+// accumulators never leave registers either.  A team is
+//   * a thread-block cluster of CL CTAs when S/16 > 1024 (L = 15, 16),
+//   * one CTA when 32 <= S/16 <= 1024,
+//   * a slice of one warp (several teams per CTA) when S/16 < 32.
+//
+// Unit tiling.  With Q = S/K^2 "units" q, unit q holds the K x K states
+//   s = (j << (L-k)) | (q << k) | b,      j, b in [0, K).
+// For fixed b the K states (over j) share the predecessor group of
+// g = (q << k) | b (the forward log-sum-exp); for fixed j the K states (over b)
+// are the successors of every state p with p & (S/K-1) == (j << (L-2k)) | q
+// (the backward log-sum-exp).  A thread holds a JT x BT tile of one unit
+// (K >= 4) or U whole units (K = 2); when K >= 8 the K/4 x K/4 tiles of a unit
+// sit in consecutive lanes and combine their partial sums with shuffles.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace bcjr {
+
+constexpr int kStatesPerThread = 16;
+
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float lg2f(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcpf(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Store v into the shared memory of CTA `rank` of this cluster at the same
+// offset as the local address `p`.
+__device__ __forceinline__ void st_cluster_f32(const float* p, uint32_t rank, float v) {
+  uint32_t a = smem_u32(p), r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(r), "f"(v) : "memory");
+}
+__device__ __forceinline__ void st_cluster_v4(const float* p, uint32_t rank, float4 v) {
+  uint32_t a = smem_u32(p), r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(r), "f"(v.x), "f"(v.y),
+               "f"(v.z), "f"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void st_cluster_f64(const double* p, uint32_t rank, double v) {
+  uint32_t a = smem_u32(p), r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+  asm volatile("st.shared::cluster.f64 [%0], %1;" ::"r"(r), "d"(v) : "memory");
+}
+__device__ __forceinline__ void st_cluster_u32(const void* p, uint32_t rank, uint32_t v) {
+  uint32_t a = smem_u32(p), r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(r), "r"(v) : "memory");
+}
+
+template <int CL>
+__device__ __forceinline__ void team_store(float* base, uint32_t rank, int off, float v) {
+  if constexpr (CL == 1) {
+    base[off] = v;
+  } else {
+    st_cluster_f32(base + off, rank, v);
+  }
+}
+template <int CL>
+__device__ __forceinline__ void team_store_f64(double* base, uint32_t rank, int off, double v) {
+  if constexpr (CL == 1) {
+    base[off] = v;
+  } else {
+    st_cluster_f64(base + off, rank, v);
+  }
+}
+template <int CL>
+__device__ __forceinline__ void team_store_u32(uint32_t* base, uint32_t rank, int off, uint32_t v) {
+  if constexpr (CL == 1) {
+    base[off] = v;
+  } else {
+    st_cluster_u32(base + off, rank, v);
+  }
+}
+
+template <int CL>
+__device__ __forceinline__ void team_sync() {
+  if constexpr (CL == 1) {
+    __syncthreads();
+  } else {
+    cluster_sync_all();
+  }
+}
+
+// Max over aligned groups of `width` lanes (width a power of two <= 32).
+__device__ __forceinline__ float group_max(float v, int width) {
+  if (width == 32) {
+    float r;
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+    return r;
+  }
+  for (int o = width >> 1; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float group_sum(float v, int width) {
+  for (int o = width >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ double group_sum_f64(double v, int width) {
+  for (int o = width >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Compile-time tile shape for 2^k predecessors.
+template <int K>
+struct Tile {
+  static constexpr int JT = K < 4 ? K : 4;                   // j values per thread
+  static constexpr int BT = K < 4 ? K : 4;                   // b values per thread
+  static constexpr int U = K <= 4 ? 16 / (K * K) : 1;        // whole units per thread
+  static constexpr int TPU = K <= 4 ? 1 : (K * K) / 16;      // threads per unit
+  static constexpr int NBT = K / BT;                         // b-tiles per unit
+  static_assert(U * JT * BT == kStatesPerThread, "16 states per thread");
+};
+
+}  // namespace bcjr
