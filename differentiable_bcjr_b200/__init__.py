@@ -40,7 +40,8 @@ class BCJRError(RuntimeError):
 
 
 class Options(ctypes.Structure):
-    _fields_ = [("checkpoint_interval", ctypes.c_int), ("reserved", ctypes.c_int * 7)]
+    _fields_ = [("checkpoint_interval", ctypes.c_int), ("sequences_in_flight", ctypes.c_int),
+                ("reserved", ctypes.c_int * 6)]
 
 
 _lib = None
@@ -79,9 +80,10 @@ def lib():
     return _lib
 
 
-def _opts(checkpoint_interval: int = 0):
+def _opts(checkpoint_interval: int = 0, sequences_in_flight: int = 0):
     o = Options()
     o.checkpoint_interval = int(checkpoint_interval)
+    o.sequences_in_flight = int(sequences_in_flight)
     return o
 
 
@@ -142,7 +144,7 @@ def get_status(ws_tensor: torch.Tensor) -> int:
 
 
 def bcjr_forward(w, codebook, T, state_bits, k, want_marginals=False, checkpoint_interval=0, ws=None,
-                 out=None):
+                 out=None, sequences_in_flight=0):
     """Soft codeword of every row of w [N][n] (float32, CUDA).  Returns
     (w_hat [N][n], marginals [N][n][S] or None, log_z [N])."""
     _need_cuda(w, codebook)
@@ -152,7 +154,7 @@ def bcjr_forward(w, codebook, T, state_bits, k, want_marginals=False, checkpoint
     w_hat = out if out is not None else torch.empty((N, n), dtype=torch.float32, device=dev)
     marg = torch.empty((N, n, S), dtype=torch.float32, device=dev) if want_marginals else None
     log_z = torch.empty((N,), dtype=torch.float32, device=dev)
-    o = _opts(checkpoint_interval)
+    o = _opts(checkpoint_interval, sequences_in_flight)
     nbytes = lib().bcjr_workspace_size(OP_FORWARD, state_bits, k, n, N, ctypes.byref(o))
     if nbytes == 0:
         raise BCJRError(2, "bcjr_workspace_size")
@@ -164,7 +166,7 @@ def bcjr_forward(w, codebook, T, state_bits, k, want_marginals=False, checkpoint
 
 
 def bcjr_backward(grad_w_hat, w, codebook, w_hat, T, state_bits, k, checkpoint_interval=0, ws=None,
-                  grad_codebook=None, accumulate_codebook=False):
+                  grad_codebook=None, accumulate_codebook=False, sequences_in_flight=0):
     """VJP of the soft codeword.  Returns (grad_w [N][n], grad_codebook [S])."""
     _need_cuda(grad_w_hat, w, codebook, w_hat)
     N, n = w.shape
@@ -174,7 +176,7 @@ def bcjr_backward(grad_w_hat, w, codebook, w_hat, T, state_bits, k, checkpoint_i
     if grad_codebook is None:
         grad_codebook = torch.empty((S,), dtype=torch.float32, device=dev)
         accumulate_codebook = False
-    o = _opts(checkpoint_interval)
+    o = _opts(checkpoint_interval, sequences_in_flight)
     nbytes = lib().bcjr_workspace_size(OP_BACKWARD, state_bits, k, n, N, ctypes.byref(o))
     if nbytes == 0:
         raise BCJRError(2, "bcjr_workspace_size")

@@ -29,6 +29,8 @@ bcjr_status check_trellis(int L, int k) {
   return BCJR_OK;
 }
 
+int seqs_in_flight(const bcjr_options* opt) { return opt ? opt->sequences_in_flight : 0; }
+
 int effective_c(const bcjr_options* opt, int n) {
   int c = (opt && opt->checkpoint_interval > 0) ? opt->checkpoint_interval : 1;
   if (c > n) c = n;
@@ -36,38 +38,48 @@ int effective_c(const bcjr_options* opt, int n) {
   return c;
 }
 
-// Byte offsets of every workspace region for one bitshift call.
+// Byte offsets of every workspace region for one bitshift call.  "Lanes" are
+// the sequences in flight: teams x sequences per team.
 struct FBLayout {
-  size_t ckpt, ckptF, ring, ringF, Mst, Cst, part, gc, total;
-  size_t ckpt_stride, ring_stride, part_stride, mc_stride;
+  size_t ck, ckF, ck64, ckF64, Mtab, Ctab, part, gc, total;
+  size_t ck_stride, ck64_stride, tab_stride, part_stride, row;
 };
+
+// Elements of one thread-private checkpoint row: (S/16 threads) x (forward
+// values per thread); k >= 3 lanes that share a forward group keep copies.
+size_t ckpt_row(int L, int k) {
+  const int K = 1 << k;
+  const int JT = K < 4 ? K : 4;
+  const int U = K <= 4 ? 16 / (K * K) : 1;
+  return (static_cast<size_t>(1) << L) / 16 * static_cast<size_t>(U * JT);
+}
 
 FBLayout fb_layout(const TeamGeometry& g, int L, int k, int n, int C, bool adjoint) {
   FBLayout l = {};
-  const size_t G = static_cast<size_t>(1) << (L - k);
-  const size_t slots = static_cast<size_t>(g.num_slots);
-  const size_t n_ckpt = static_cast<size_t>((n - 1) / C + 1);
-  l.ckpt_stride = n_ckpt * G;
-  l.ring_stride = C > 1 ? static_cast<size_t>(C) * G : 0;
+  const size_t row = ckpt_row(L, k);
+  const size_t lanes = static_cast<size_t>(g.num_slots) * g.nseq;
+  l.row = row;
+  l.ck_stride = (C == 1 ? static_cast<size_t>(n) : static_cast<size_t>(C)) * row;
+  l.ck64_stride = C == 1 ? 0 : static_cast<size_t>((n - 1) / C + 1) * row;
+  l.tab_stride = static_cast<size_t>(n) + 1;
   l.part_stride = static_cast<size_t>(n) * 2 * g.warps_per_team;
-  l.mc_stride = static_cast<size_t>(n) + 1;
   size_t off = kHeaderBytes;
-  l.ckpt = off;
-  off = align_up(off + slots * l.ckpt_stride * sizeof(float));
-  l.ckptF = off;
-  if (adjoint) off = align_up(off + slots * l.ckpt_stride * sizeof(float));
-  l.ring = off;
-  off = align_up(off + slots * l.ring_stride * sizeof(float));
-  l.ringF = off;
-  if (adjoint) off = align_up(off + slots * l.ring_stride * sizeof(float));
-  l.Mst = off;
-  off = align_up(off + slots * l.mc_stride * sizeof(float));
-  l.Cst = off;
-  off = align_up(off + slots * l.mc_stride * sizeof(double));
+  l.ck = off;
+  off = align_up(off + lanes * l.ck_stride * sizeof(float));
+  l.ckF = off;
+  if (adjoint) off = align_up(off + lanes * l.ck_stride * sizeof(float));
+  l.ck64 = off;
+  off = align_up(off + lanes * l.ck64_stride * sizeof(double));
+  l.ckF64 = off;
+  if (adjoint) off = align_up(off + lanes * l.ck64_stride * sizeof(float));
+  l.Mtab = off;
+  off = align_up(off + lanes * l.tab_stride * sizeof(float));
+  l.Ctab = off;
+  off = align_up(off + lanes * l.tab_stride * sizeof(double));
   l.part = off;
-  off = align_up(off + slots * l.part_stride * sizeof(float));
+  off = align_up(off + lanes * l.part_stride * sizeof(float));
   l.gc = off;
-  if (adjoint) off = align_up(off + slots * (static_cast<size_t>(1) << L) * sizeof(float));
+  if (adjoint) off = align_up(off + static_cast<size_t>(g.num_slots) * (static_cast<size_t>(1) << L) * sizeof(float));
   l.total = off;
   return l;
 }
@@ -128,8 +140,9 @@ size_t bcjr_workspace_size(int op, int state_bits, int k, int seq_len, int n_seq
   TeamGeometry g;
   if (op == BCJR_OP_FORWARD || op == BCJR_OP_BACKWARD) {
     const bool adj = op == BCJR_OP_BACKWARD;
-    if (bcjr::fb_geometry(state_bits, k, nq, adj, &g) != cudaSuccess) return 0;
-    return fb_layout(g, state_bits, k, seq_len, effective_c(opt, seq_len), adj).total;
+    const int C = effective_c(opt, seq_len);
+    if (bcjr::fb_geometry(state_bits, k, nq, adj, C, seqs_in_flight(opt), &g) != cudaSuccess) return 0;
+    return fb_layout(g, state_bits, k, seq_len, C, adj).total;
   }
   if (op == BCJR_OP_VITERBI) {
     if (bcjr::viterbi_geometry(state_bits, k, nq, &g) != cudaSuccess) return 0;
@@ -145,7 +158,8 @@ static bcjr_status fb_common(bool adjoint, const float* grad_w_hat, const float*
   bcjr_status st = check_trellis(L, k);
   if (st != BCJR_OK) return st;
   if (n < 1 || N < 0 || !(T > 0.f) || !std::isfinite(T)) return BCJR_ERR_INVALID_ARG;
-  if (opt && opt->checkpoint_interval < 0) return BCJR_ERR_INVALID_ARG;
+  if (opt && (opt->checkpoint_interval < 0 || opt->sequences_in_flight < 0 || opt->sequences_in_flight > 1))
+    return BCJR_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int S = 1 << L;
   if (N == 0) {  // no sequences: the per-sequence arrays may be empty (null)
@@ -161,8 +175,8 @@ static bcjr_status fb_common(bool adjoint, const float* grad_w_hat, const float*
   }
   if (!ws || !aligned(ws, kAlign)) return BCJR_ERR_WORKSPACE;
   TeamGeometry g;
-  if ((st = from_cuda(bcjr::fb_geometry(L, k, N, adjoint, &g))) != BCJR_OK) return st;
   const int C = effective_c(opt, n);
+  if ((st = from_cuda(bcjr::fb_geometry(L, k, N, adjoint, C, seqs_in_flight(opt), &g))) != BCJR_OK) return st;
   const FBLayout lay = fb_layout(g, L, k, n, C, adjoint);
   if (ws_bytes < lay.total) return BCJR_ERR_WORKSPACE;
   char* base = static_cast<char*>(ws);
@@ -176,19 +190,20 @@ static bcjr_status fb_common(bool adjoint, const float* grad_w_hat, const float*
   p.log_z = log_z;
   p.grad_w = grad_w;
   p.gc_part = reinterpret_cast<float*>(base + lay.gc);
-  p.ckpt = reinterpret_cast<float*>(base + lay.ckpt);
-  p.ckptF = reinterpret_cast<float*>(base + lay.ckptF);
-  p.ring = reinterpret_cast<float*>(base + lay.ring);
-  p.ringF = reinterpret_cast<float*>(base + lay.ringF);
-  p.Mst = reinterpret_cast<float*>(base + lay.Mst);
-  p.Cst = reinterpret_cast<double*>(base + lay.Cst);
+  p.ck = reinterpret_cast<float*>(base + lay.ck);
+  p.ckF = reinterpret_cast<float*>(base + lay.ckF);
+  p.ck64 = reinterpret_cast<double*>(base + lay.ck64);
+  p.ckF64 = reinterpret_cast<float*>(base + lay.ckF64);
+  p.Mtab = reinterpret_cast<float*>(base + lay.Mtab);
+  p.Ctab = reinterpret_cast<double*>(base + lay.Ctab);
   p.part = reinterpret_cast<float*>(base + lay.part);
   p.status = reinterpret_cast<int*>(base);
-  p.ckpt_stride = lay.ckpt_stride;
-  p.ring_stride = lay.ring_stride;
+  p.ck_stride = lay.ck_stride;
+  p.ck64_stride = lay.ck64_stride;
+  p.tab_stride = lay.tab_stride;
   p.part_stride = lay.part_stride;
-  p.mc_stride = lay.mc_stride;
-  p.sc = static_cast<float>(1.4426950408889634 / static_cast<double>(T));
+  p.row = lay.row;
+  p.sc64 = 1.4426950408889634 / static_cast<double>(T);
   p.two_over_T = static_cast<float>(2.0 / static_cast<double>(T));
   p.L = L;
   p.k = k;

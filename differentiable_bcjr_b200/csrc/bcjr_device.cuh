@@ -50,7 +50,12 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   return r;
 }
 
+// The .aligned cluster barriers require every lane of the warp to execute
+// them together; lanes that ran a divergent branch just before (e.g. lane 0
+// publishing a warp result) are re-joined first, so that their stores precede
+// the warp's arrival.
 __device__ __forceinline__ void cluster_sync_all() {
+  __syncwarp();
   asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
                "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
@@ -143,5 +148,40 @@ struct Tile {
   static constexpr int NBT = K / BT;                         // b-tiles per unit
   static_assert(U * JT * BT == kStatesPerThread, "16 states per thread");
 };
+
+}  // namespace bcjr
+
+namespace bcjr {
+
+__device__ __forceinline__ void st_cluster_v2f64(const double* p, uint32_t rank, double a, double b) {
+  uint32_t addr = smem_u32(p), r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  asm volatile("st.shared::cluster.v2.f64 [%0], {%1, %2};" ::"r"(r), "d"(a), "d"(b) : "memory");
+}
+
+// Split cluster barrier: arrive (release) now, wait (acquire) later.
+__device__ __forceinline__ void cluster_arrive() {
+  __syncwarp();
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  __syncwarp();
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Asynchronous 16-byte global -> shared copy, completed with cp_async_wait<N>.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ double group_max_f64(double v, int width) {
+  for (int o = width >> 1; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
 
 }  // namespace bcjr

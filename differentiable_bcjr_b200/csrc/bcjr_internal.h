@@ -19,6 +19,7 @@ struct TeamGeometry {
   int block_threads;   // threads per CTA
   int teams_per_cta;   // > 1 only when a team is narrower than a warp
   int warps_per_team;  // max(1, team_threads / 32)
+  int nseq;            // sequences in flight per team (forward-backward kernels)
   int num_slots;       // teams resident in the grid (persistent)
   int grid_blocks;
   size_t smem_bytes;   // dynamic shared memory per CTA
@@ -34,23 +35,62 @@ struct FBParams {
   float* log_z;            // [N] or null (forward)
   float* grad_w;           // [N][n] (backward)
   float* gc_part;          // [slots][S] per-team codebook-gradient partials (backward)
-  float* ckpt;             // per slot [n_ckpt][G]: raw forward group vectors every C steps
-  float* ckptF;            // per slot [n_ckpt][G]: forward adjoint accumulators (backward)
-  float* ring;             // per slot [C][G]: recomputed segment (C > 1)
-  float* ringF;            // per slot [C][G]
-  float* Mst;              // per slot [n + 1]: per-step maxima used to rescale
-  double* Cst;             // per slot [n + 1]: accumulated forward log2 scale
-  float* part;             // per slot [n][2][warps_per_team]: per-warp partial sums
+  // Per sequence in flight ("lane" = slot * nseq + x).  Rows are thread-private:
+  // thread tt of the team owns elements [tt*NV, tt*NV + NV) of every row, so a
+  // row holds team_threads * NV values (= S/2^k for k <= 2, S/4 for k >= 3,
+  // where lanes sharing a forward group each keep their own copy).
+  float* ck;               // C == 1: [n][row] forward values A_t - M_t (float); C > 1: ring [C][row]
+  float* ckF;              // same for the forward adjoint accumulators (backward)
+  double* ck64;            // C > 1: [n/C + 1][row] A_t - M_t at t = 0, C, 2C, ... (float64)
+  float* ckF64;            // C > 1: [n/C + 1][row] forward adjoint accumulators at the same t
+  float* Mtab;             // [n + 1] team max M_t of the raw forward vector
+  double* Ctab;            // [n + 1] log2 scale C_{t+1} = C_t + M_t of the forward vector
+  float* part;             // [n][2][warps_per_team] per-warp partial sums
   int* status;
-  size_t ckpt_stride;      // floats per slot in ckpt / ckptF
-  size_t ring_stride;      // floats per slot in ring / ringF
-  size_t part_stride;      // floats per slot in part
-  size_t mc_stride;        // entries per slot in Mst / Cst
-  float sc;                // log2(e) / T
+  size_t ck_stride;        // floats per lane in ck / ckF
+  size_t ck64_stride;      // elements per lane in ck64 / ckF64
+  size_t tab_stride;       // entries per lane in Mtab / Ctab
+  size_t part_stride;      // floats per lane in part
+  size_t row;              // elements per checkpoint row (team_threads * NV)
+  double sc64;             // log2(e) / T
   float two_over_T;
   int L, k, n, N, C;
   int num_slots;
 };
+
+// Shared-memory carve-up of the forward-backward kernel (bytes), identical on
+// host and device.  Per team and per sequence in flight: the double-buffered
+// exchange vectors (float64 group values, float32 adjoint accumulators) and
+// the per-warp maxima; per CTA: a reduction scratch and the thread-private
+// staging of the forward values read by the backward sweep.
+struct FBSmem {
+  uint32_t exA, exF, exB, exBt, maxp, per_seq, per_team, red, stage, stageF, total;
+};
+__host__ __device__ inline FBSmem fb_smem_layout(int GL, int NT, int NV, int nseq, bool adj, bool alias,
+                                                 int teams_per_cta) {
+  FBSmem l;
+  uint32_t o = 0;
+  l.exA = o;
+  o += 2u * GL * 8u;
+  l.exF = o;
+  if (adj) o += 2u * GL * 4u;
+  l.exB = alias ? l.exA : o;
+  if (!alias) o += 2u * GL * 8u;
+  l.exBt = alias ? l.exF : o;
+  if (!alias && adj) o += 2u * GL * 4u;
+  l.maxp = o;
+  o += 2u * 128u * 4u;
+  l.per_seq = o;
+  l.per_team = static_cast<uint32_t>(nseq) * o;
+  l.red = static_cast<uint32_t>(teams_per_cta) * l.per_team;
+  o = l.red + 4u * 128u * 4u;
+  l.stage = o;
+  o += static_cast<uint32_t>(nseq) * 2u * NT * NV * 4u;
+  l.stageF = o;
+  if (adj) o += static_cast<uint32_t>(nseq) * 2u * NT * NV * 4u;
+  l.total = o;
+  return l;
+}
 
 struct ViterbiParams {
   const float* w;
@@ -70,9 +110,9 @@ cudaError_t launch_fb(const FBParams& p, const TeamGeometry& g, bool adjoint, cu
 cudaError_t launch_viterbi(const ViterbiParams& p, const TeamGeometry& g, cudaStream_t s);
 cudaError_t launch_gradc_reduce(const float* gc_part, int num_slots, int S, float* grad_c,
                                 int accumulate, cudaStream_t s);
-// Host-side geometry: fills everything except num_slots/grid_blocks when
-// `occupancy` is false; with it, also the persistent grid for this device.
-cudaError_t fb_geometry(int L, int k, int n_seq, bool adjoint, TeamGeometry* g);
+// Host-side geometry and persistent grid for this device.  cudaErrorNotSupported
+// when no configuration fits the shared memory of one CTA.
+cudaError_t fb_geometry(int L, int k, int n_seq, bool adjoint, int C, int nseq_request, TeamGeometry* g);
 cudaError_t viterbi_geometry(int L, int k, int n_seq, TeamGeometry* g);
 
 }  // namespace bcjr

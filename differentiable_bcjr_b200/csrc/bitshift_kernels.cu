@@ -1,572 +1,23 @@
-// bitshift_kernels.cu -- BCJR forward-backward over the bitshift trellis on sm_100a.
+// bitshift_kernels.cu -- hard decode, codebook-gradient reduction, and the host-side
+// geometry and launches of the bitshift-trellis kernels (sm_100a).
 //
-// "BCJR-QAT: A Differentiable Relaxation of Trellis-Coded Weight Quantization",
-// technical summary, "core mechanism": the soft codeword
-//     w_hat_t = sum_s c(s) p_T(s_t = s | w)
-// is the Boltzmann expectation of the emitted codeword under the path
-// distribution at temperature T; "key technical innovations": the forward-
-// backward recursion gives exact gradients through the trellis, and the
-// pages' own kernel fuses gather, log-sum-exp and add into one launch.
-//
-// Trellis (bitshift): pred(s) = {(j << (L-k)) | (s >> k) : j < K}, K = 2^k.
-// Emission log-weight phi_t(s) = -(w_t - c(s))^2 / T; uniform start; free end.
-//
-// Group form used here (exact rewrite of the forward-backward):
-//   alpha_t(s) = phi_t(s) + A_t(s >> k),   A_{t+1}(g) = LSE_j alpha_t((j << (L-k)) | g)
-//   beta_t(p)  = B_t(p & (S/K - 1)),       B_{t-1}(h) = LSE_b [phi_t((h << k) | b) + B_t(((h << k) | b) & (S/K - 1))]
-// so a sweep step is one K-term log-sum-exp per group of K states, and only
-// the S/K group values travel between threads.  Everything is computed in
-// base 2 (phi scaled by log2 e); every step subtracts the exact team-wide
-// maximum of the incoming group vector and the shift is carried in float64.
-//
-// One launch does a whole call: the forward sweep (storing the raw group
-// vector every C steps), then the backward sweep (recomputing the missing
-// steps of each C-segment), then the per-step reductions of the outputs.
+// The fused forward-backward kernel itself is fb_kernel.cuh, instantiated per k
+// in fb_fwd_k*.cu / fb_adj_k*.cu.
 #include <cfloat>
 #include <cmath>
+#include <map>
+#include <mutex>
+#include <tuple>
 
 #include "bcjr_device.cuh"
 #include "bcjr_internal.h"
+#include "team.cuh"
 
 namespace bcjr {
 
 namespace {
-
-constexpr float kNegInf = -INFINITY;
 constexpr unsigned kFull = 0xffffffffu;
-
-// Per-thread state shared by the sweeps of one launch.
-template <int K, int CL>
-struct Team {
-  using TL = Tile<K>;
-  int L, k, S, G, Q, TS, GL, Qc;
-  int tt, lane, width, wpt, warp_in_team;
-  uint32_t rank;
-  int q0, j0, b0, qloc0;
-  bool a_writer, b_writer;
-
-  __device__ void init(int L_, int k_, int team_in_cta_threads_offset) {
-    L = L_;
-    k = k_;
-    S = 1 << L;
-    G = S >> k;
-    Q = S >> (2 * k);
-    TS = S / kStatesPerThread;
-    GL = G / CL;
-    Qc = Q / CL;
-    lane = threadIdx.x & 31;
-    if constexpr (CL > 1) {
-      rank = cluster_rank();
-      tt = static_cast<int>(rank) * blockDim.x + threadIdx.x;
-    } else {
-      rank = 0;
-      tt = threadIdx.x - team_in_cta_threads_offset;
-    }
-    width = TS < 32 ? TS : 32;
-    wpt = TS < 32 ? 1 : TS / 32;
-    warp_in_team = TS < 32 ? 0 : (tt >> 5);
-    if constexpr (K <= 4) {
-      q0 = tt * TL::U;
-      j0 = 0;
-      b0 = 0;
-    } else {
-      q0 = tt / TL::TPU;
-      const int tile = tt % TL::TPU;
-      j0 = 4 * (tile / TL::NBT);
-      b0 = 4 * (tile % TL::NBT);
-    }
-    qloc0 = q0 - static_cast<int>(rank) * Qc;
-    a_writer = (j0 == 0);
-    b_writer = (b0 == 0);
-  }
-  __device__ __forceinline__ int state(int u, int jj, int bb) const {
-    return ((j0 + jj) << (L - k)) | ((q0 + u) << k) | (b0 + bb);
-  }
-  // Forward-sweep layout: value index i lives with the unit that reads it.
-  __device__ __forceinline__ int a_read_off(int u, int jj) const { return (j0 + jj) * Qc + qloc0 + u; }
-  __device__ __forceinline__ void a_dest(int g, uint32_t& r, int& off) const {
-    const int qq = g & (Q - 1), jj = g >> (L - 2 * k);
-    r = static_cast<uint32_t>(qq / Qc);
-    off = jj * Qc + (qq - static_cast<int>(r) * Qc);
-  }
-  // Backward-sweep layout: contiguous blocks of G/CL values per CTA.
-  __device__ __forceinline__ int b_read_off(int u, int bb) const { return (qloc0 + u) * K + b0 + bb; }
-  __device__ __forceinline__ void b_dest(int h, uint32_t& r, int& off) const {
-    r = static_cast<uint32_t>(h / GL);
-    off = h - static_cast<int>(r) * GL;
-  }
-  // Output index of the forward step (group of successors) and of the backward step.
-  __device__ __forceinline__ int a_out_index(int u, int bb) const { return ((q0 + u) << k) | (b0 + bb); }
-  __device__ __forceinline__ int b_out_index(int u, int jj) const {
-    return ((j0 + jj) << (L - 2 * k)) | (q0 + u);
-  }
-};
-
-// Team-wide maximum of one value per thread, published through shared memory
-// of every CTA of the team; read back after the next team barrier.
-template <int K, int CL>
-__device__ __forceinline__ float publish_max(const Team<K, CL>& tm, float* maxp_buf, float v) {
-  const float wm = group_max(v, tm.width);
-  if (tm.TS > 32 && tm.lane == 0) {
-#pragma unroll
-    for (int r = 0; r < CL; ++r) team_store<CL>(maxp_buf, r, tm.warp_in_team, wm);
-  }
-  return wm;
-}
-template <int K, int CL>
-__device__ __forceinline__ float collect_max(const Team<K, CL>& tm, const float* maxp_buf, float wm) {
-  if (tm.TS <= 32) return wm;
-  float m = kNegInf;
-  for (int i = tm.lane; i < tm.wpt; i += 32) m = fmaxf(m, maxp_buf[i]);
-  return group_max(m, 32);
-}
-
-// Team-wide sum (fixed order, so every thread gets the same bits).
-template <int K, int CL>
-__device__ __forceinline__ float team_sum(const Team<K, CL>& tm, float* red, float v) {
-  v = group_sum(v, tm.width);
-  if (tm.TS <= 32) return v;
-  if (tm.lane == 0) {
-#pragma unroll
-    for (int r = 0; r < CL; ++r) team_store<CL>(red, r, tm.warp_in_team, v);
-  }
-  team_sync<CL>();
-  float s = 0.f;
-  for (int i = 0; i < tm.wpt; ++i) s += red[i];
-  team_sync<CL>();
-  return s;
-}
-
-// One forward step for the thread's states: inputs a[u][jj] = normalised
-// group values A_t of the predecessor groups (f: adjoint accumulators),
-// outputs the raw A_{t+1} of the thread's output groups (fo: accumulators).
-//   adjoint accumulator  F_{t+1}(g) = sum_j pi_j (F_t(p_j >> k) + g_t (c(p_j) - w_hat_t)),
-//   pi_j = the forward log-sum-exp's own softmax weights.
-template <int K, bool ADJ>
-__device__ __forceinline__ void forward_step(const float (&cb)[Tile<K>::U][Tile<K>::JT][Tile<K>::BT],
-                                             float wt, float sc, float gt, float gw,
-                                             const float (&a)[Tile<K>::U][Tile<K>::JT],
-                                             const float (&f)[Tile<K>::U][Tile<K>::JT],
-                                             float (&out)[Tile<K>::U][Tile<K>::BT],
-                                             float (&fo)[Tile<K>::U][Tile<K>::BT]) {
-  using TL = Tile<K>;
-#pragma unroll
-  for (int u = 0; u < TL::U; ++u) {
-#pragma unroll
-    for (int bb = 0; bb < TL::BT; ++bb) {
-      float x[TL::JT];
-      float m = kNegInf;
-#pragma unroll
-      for (int jj = 0; jj < TL::JT; ++jj) {
-        const float d = wt - cb[u][jj][bb];
-        x[jj] = fmaf(-sc * d, d, a[u][jj]);
-        m = fmaxf(m, x[jj]);
-      }
-      if constexpr (K >= 8) {
-#pragma unroll
-        for (int o = TL::NBT; o < TL::TPU; o <<= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-      }
-      float s = 0.f, num = 0.f;
-#pragma unroll
-      for (int jj = 0; jj < TL::JT; ++jj) {
-        const float e = ex2f(x[jj] - m);
-        s += e;
-        if constexpr (ADJ) num = fmaf(e, f[u][jj] + fmaf(gt, cb[u][jj][bb], -gw), num);
-      }
-      if constexpr (K >= 8) {
-#pragma unroll
-        for (int o = TL::NBT; o < TL::TPU; o <<= 1) {
-          s += __shfl_xor_sync(kFull, s, o);
-          if constexpr (ADJ) num += __shfl_xor_sync(kFull, num, o);
-        }
-      }
-      out[u][bb] = m + lg2f(s);
-      if constexpr (ADJ) fo[u][bb] = num * rcpf(s);
-    }
-  }
-}
-
-template <bool ADJ>
-__host__ __device__ constexpr size_t fb_smem_floats_per_team(int GL) {
-  return static_cast<size_t>(ADJ ? 8 : 4) * GL + 2 * 128 + 4 * 128;
-}
-
 }  // namespace
-
-template <int K, int CL, bool ADJ, int NTB>
-__global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
-  using TL = Tile<K>;
-  constexpr int U = TL::U, JT = TL::JT, BT = TL::BT;
-  const int L = p.L, k = p.k, n = p.n;
-  const int S = 1 << L;
-  const int TS = S / kStatesPerThread;
-  const int tpc = (CL == 1 && TS < static_cast<int>(blockDim.x)) ? static_cast<int>(blockDim.x) / TS : 1;
-  const int team_in_cta = (tpc > 1) ? static_cast<int>(threadIdx.x) / TS : 0;
-  Team<K, CL> tm;
-  tm.init(L, k, team_in_cta * TS);
-  const int slot = (CL > 1) ? static_cast<int>(blockIdx.x) / CL : static_cast<int>(blockIdx.x) * tpc + team_in_cta;
-  const int G = tm.G, GL = tm.GL;
-
-  extern __shared__ __align__(16) float smem[];
-  float* base = smem + team_in_cta * fb_smem_floats_per_team<ADJ>(GL);
-  float* bufA = base;
-  float* bufF = bufA + 2 * GL;
-  float* bufB = bufA + (ADJ ? 4 : 2) * GL;
-  float* bufBt = bufB + 2 * GL;
-  float* maxp = bufA + (ADJ ? 8 : 4) * GL;
-  float* red = maxp + 2 * 128;
-
-  float cb[U][JT][BT];
-#pragma unroll
-  for (int u = 0; u < U; ++u)
-#pragma unroll
-    for (int jj = 0; jj < JT; ++jj)
-#pragma unroll
-      for (int bb = 0; bb < BT; ++bb) cb[u][jj][bb] = __ldg(p.codebook + tm.state(u, jj, bb));
-
-  float gc[U][JT][BT];
-  if constexpr (ADJ) {
-#pragma unroll
-    for (int u = 0; u < U; ++u)
-#pragma unroll
-      for (int jj = 0; jj < JT; ++jj)
-#pragma unroll
-        for (int bb = 0; bb < BT; ++bb) gc[u][jj][bb] = 0.f;
-  }
-
-  float* ckpt = p.ckpt + static_cast<size_t>(slot) * p.ckpt_stride;
-  float* ckptF = ADJ ? p.ckptF + static_cast<size_t>(slot) * p.ckpt_stride : nullptr;
-  float* ring = p.C > 1 ? p.ring + static_cast<size_t>(slot) * p.ring_stride : nullptr;
-  float* ringF = (ADJ && p.C > 1) ? p.ringF + static_cast<size_t>(slot) * p.ring_stride : nullptr;
-  float* Mst = p.Mst + static_cast<size_t>(slot) * p.mc_stride;
-  double* Cst = p.Cst + static_cast<size_t>(slot) * p.mc_stride;
-  float* part = p.part + static_cast<size_t>(slot) * p.part_stride;
-  const int C = p.C;
-  const float sc = p.sc;
-
-  const int iters = (p.N + p.num_slots - 1) / p.num_slots;
-  for (int it = 0; it < iters; ++it) {
-    const int seq_raw = slot + it * p.num_slots;
-    const bool active = seq_raw < p.N;
-    const int seq = active ? seq_raw : p.N - 1;
-    const float* wseq = p.w + static_cast<size_t>(seq) * n;
-    const float* gseq = ADJ ? p.g + static_cast<size_t>(seq) * n : nullptr;
-    const float* hseq = ADJ ? p.what_in + static_cast<size_t>(seq) * n : nullptr;
-
-    // ------------------------------------------------------------------
-    // Forward sweep: t = 0 .. n-1 produces raw A_{t+1}; A_0 = 0.
-    // ------------------------------------------------------------------
-    float Mt = 0.f;   // max of raw A_t (team-wide); subtracted on read
-    double Ct = 0.0;  // A_t(true) = raw A_t + C_t  (log2 units)
-    float out[U][BT], fo[U][BT];
-    for (int t = 0; t < n; ++t) {
-      const float wt = __ldg(wseq + t);
-      float gt = 0.f, gw = 0.f;
-      if constexpr (ADJ) {
-        gt = __ldg(gseq + t);
-        gw = gt * __ldg(hseq + t);
-      }
-      float a[U][JT], f[U][JT];
-      const float* rA = bufA + (t & 1) * GL;
-      const float* rF = bufF + (t & 1) * GL;
-#pragma unroll
-      for (int u = 0; u < U; ++u)
-#pragma unroll
-        for (int jj = 0; jj < JT; ++jj) {
-          a[u][jj] = (t == 0) ? 0.f : rA[tm.a_read_off(u, jj)] - Mt;
-          if constexpr (ADJ) f[u][jj] = (t == 0) ? 0.f : rF[tm.a_read_off(u, jj)];
-        }
-      forward_step<K, ADJ>(cb, wt, sc, gt, gw, a, f, out, fo);
-      float lmax = kNegInf;
-      if (tm.a_writer) {
-        const bool keep = (t + 1 < n) && ((t + 1) % C == 0);
-        float* crow = ckpt + static_cast<size_t>((t + 1) / C) * G;
-        float* crowF = ADJ ? ckptF + static_cast<size_t>((t + 1) / C) * G : nullptr;
-#pragma unroll
-        for (int u = 0; u < U; ++u)
-#pragma unroll
-          for (int bb = 0; bb < BT; ++bb) {
-            lmax = fmaxf(lmax, out[u][bb]);
-            if (t + 1 < n) {
-              const int gi = tm.a_out_index(u, bb);
-              uint32_t r;
-              int off;
-              tm.a_dest(gi, r, off);
-              team_store<CL>(bufA + ((t + 1) & 1) * GL, r, off, out[u][bb]);
-              if constexpr (ADJ) team_store<CL>(bufF + ((t + 1) & 1) * GL, r, off, fo[u][bb]);
-              if (keep) {
-                crow[gi] = out[u][bb];
-                if constexpr (ADJ) crowF[gi] = fo[u][bb];
-              }
-            }
-          }
-      }
-      const float wm = publish_max(tm, maxp + ((t + 1) & 1) * 128, lmax);
-      if (tm.tt == 0) {
-        Mst[t] = Mt;
-        Cst[t] = Ct;
-      }
-      team_sync<CL>();
-      const float Mn = collect_max(tm, maxp + ((t + 1) & 1) * 128, wm);
-      Ct += static_cast<double>(Mt);
-      Mt = Mn;
-    }
-    // Now out = raw A_n (never stored), Mt = max A_n, Ct = C_n.
-    // log2 Z = C_n + log2 sum_g 2^{A_n(g)};  D = E[sum_t g_t (c(s_t) - w_hat_t)].
-    float s1 = 0.f, s2 = 0.f;
-    if (tm.a_writer) {
-#pragma unroll
-      for (int u = 0; u < U; ++u)
-#pragma unroll
-        for (int bb = 0; bb < BT; ++bb) {
-          const float e = ex2f(out[u][bb] - Mt);
-          s1 += e;
-          if constexpr (ADJ) s2 = fmaf(e, fo[u][bb], s2);
-        }
-    }
-    s1 = team_sum(tm, red, s1);
-    if constexpr (ADJ) s2 = team_sum(tm, red + 128, s2);
-    const double log2Z = Ct + static_cast<double>(Mt) + log2(static_cast<double>(s1));
-    const float Dc = ADJ ? s2 / s1 : 0.f;
-    if (tm.tt == 0 && active) {
-      if (!isfinite(log2Z)) atomicOr(p.status, kDevNonFinite);
-      if constexpr (!ADJ) {
-        if (p.log_z) p.log_z[seq] = static_cast<float>(log2Z * 0.69314718055994530942);
-      }
-    }
-
-    // ------------------------------------------------------------------
-    // Backward sweep: t = n-1 .. 0 consumes B_t, produces raw B_{t-1}.
-    // ------------------------------------------------------------------
-    float Mb = 0.f;
-    double Dt = 0.0;  // B_t(true) = raw B_t + D_t
-    for (int t = n - 1; t >= 0; --t) {
-      // Recompute the forward group vectors of this C-segment when they were not kept.
-      if (C > 1 && t >= 1 && (t == n - 1 || (t + 1) % C == 0)) {
-        const int t0 = t - (t % C);
-        for (int tp = t0; tp < t; ++tp) {
-          const float wt = __ldg(wseq + tp);
-          float gt = 0.f, gw = 0.f;
-          if constexpr (ADJ) {
-            gt = __ldg(gseq + tp);
-            gw = gt * __ldg(hseq + tp);
-          }
-          const float Mtp = Mst[tp];
-          float a[U][JT], f[U][JT];
-          const float* crow = ckpt + static_cast<size_t>(t0 / C) * G;
-          const float* crowF = ADJ ? ckptF + static_cast<size_t>(t0 / C) * G : nullptr;
-#pragma unroll
-          for (int u = 0; u < U; ++u)
-#pragma unroll
-            for (int jj = 0; jj < JT; ++jj) {
-              const int gi = ((tm.j0 + jj) << (L - 2 * k)) | (tm.q0 + u);
-              float av, fv = 0.f;
-              if (tp == 0) {
-                av = 0.f;
-              } else if (tp == t0) {
-                av = crow[gi] - Mtp;
-                if constexpr (ADJ) fv = crowF[gi];
-              } else {
-                av = bufA[(tp & 1) * GL + tm.a_read_off(u, jj)] - Mtp;
-                if constexpr (ADJ) fv = bufF[(tp & 1) * GL + tm.a_read_off(u, jj)];
-              }
-              a[u][jj] = av;
-              if constexpr (ADJ) f[u][jj] = fv;
-            }
-          float ro[U][BT], rfo[U][BT];
-          forward_step<K, ADJ>(cb, wt, sc, gt, gw, a, f, ro, rfo);
-          if (tm.a_writer) {
-            float* rrow = ring + static_cast<size_t>(tp + 1 - t0) * G;
-            float* rrowF = ADJ ? ringF + static_cast<size_t>(tp + 1 - t0) * G : nullptr;
-#pragma unroll
-            for (int u = 0; u < U; ++u)
-#pragma unroll
-              for (int bb = 0; bb < BT; ++bb) {
-                const int gi = tm.a_out_index(u, bb);
-                uint32_t r;
-                int off;
-                tm.a_dest(gi, r, off);
-                team_store<CL>(bufA + ((tp + 1) & 1) * GL, r, off, ro[u][bb]);
-                rrow[gi] = ro[u][bb];
-                if constexpr (ADJ) {
-                  team_store<CL>(bufF + ((tp + 1) & 1) * GL, r, off, rfo[u][bb]);
-                  rrowF[gi] = rfo[u][bb];
-                }
-              }
-          }
-          team_sync<CL>();
-        }
-      }
-
-      const float wt = __ldg(wseq + t);
-      float gt = 0.f, gw = 0.f;
-      if constexpr (ADJ) {
-        gt = __ldg(gseq + t);
-        gw = gt * __ldg(hseq + t);
-      }
-      // Incoming backward group values B_t (normalised) at (q << k) | b.
-      float bv[U][BT], btl[U][BT];
-      const float* rB = bufB + (t & 1) * GL;
-      const float* rBt = bufBt + (t & 1) * GL;
-#pragma unroll
-      for (int u = 0; u < U; ++u)
-#pragma unroll
-        for (int bb = 0; bb < BT; ++bb) {
-          bv[u][bb] = (t == n - 1) ? 0.f : rB[tm.b_read_off(u, bb)] - Mb;
-          if constexpr (ADJ) btl[u][bb] = (t == n - 1) ? 0.f : rBt[tm.b_read_off(u, bb)];
-        }
-      // Forward group values A_t at the groups h = (j << (L-2k)) | q of the thread's states.
-      float ra[U][JT], fa[U][JT];
-      {
-        const float* row = nullptr;
-        const float* rowF = nullptr;
-        if (t >= 1) {
-          if (C == 1 || t % C == 0) {
-            row = ckpt + static_cast<size_t>(t / C) * G;
-            if constexpr (ADJ) rowF = ckptF + static_cast<size_t>(t / C) * G;
-          } else {
-            row = ring + static_cast<size_t>(t % C) * G;
-            if constexpr (ADJ) rowF = ringF + static_cast<size_t>(t % C) * G;
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u)
-#pragma unroll
-          for (int jj = 0; jj < JT; ++jj) {
-            const int h = tm.b_out_index(u, jj);
-            ra[u][jj] = (t >= 1) ? row[h] : 0.f;
-            if constexpr (ADJ) fa[u][jj] = (t >= 1) ? rowF[h] : 0.f;
-          }
-      }
-      // gamma_t(s) = 2^{y_b - m + m + A_t(h) + C_t + Mb + D_t - log2 Z}
-      const float kap = static_cast<float>(static_cast<double>(Mb) + Cst[t] + Dt - log2Z);
-      const float tw = p.two_over_T * wt;
-      float acc0 = 0.f, acc1 = 0.f;  // forward: sum c gamma, sum gamma; backward: sum psi c
-      float bo[U][JT], bto[U][JT];
-      float* mrow = (!ADJ && p.marginals && active)
-                        ? p.marginals + (static_cast<size_t>(seq) * n + t) * static_cast<size_t>(S)
-                        : nullptr;
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-#pragma unroll
-        for (int jj = 0; jj < JT; ++jj) {
-          float y[BT];
-          float m = kNegInf;
-#pragma unroll
-          for (int bb = 0; bb < BT; ++bb) {
-            const float d = wt - cb[u][jj][bb];
-            y[bb] = fmaf(-sc * d, d, bv[u][bb]);
-            m = fmaxf(m, y[bb]);
-          }
-          if constexpr (K >= 8) {
-#pragma unroll
-            for (int o = 1; o < TL::NBT; o <<= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
-          }
-          float e[BT];
-          float s = 0.f, ec = 0.f, bnum = 0.f;
-          float eps[BT];
-#pragma unroll
-          for (int bb = 0; bb < BT; ++bb) {
-            e[bb] = ex2f(y[bb] - m);
-            s += e[bb];
-            ec = fmaf(e[bb], cb[u][jj][bb], ec);
-            if constexpr (ADJ) {
-              eps[bb] = fmaf(gt, cb[u][jj][bb], -gw) + btl[u][bb];
-              bnum = fmaf(e[bb], eps[bb], bnum);
-            }
-          }
-          const float s_own = s;
-          if constexpr (K >= 8) {
-#pragma unroll
-            for (int o = 1; o < TL::NBT; o <<= 1) {
-              s += __shfl_xor_sync(kFull, s, o);
-              if constexpr (ADJ) bnum += __shfl_xor_sync(kFull, bnum, o);
-            }
-          }
-          bo[u][jj] = m + lg2f(s);
-          if constexpr (ADJ) bto[u][jj] = bnum * rcpf(s);
-          const float Gf = ex2f(m + ra[u][jj] + kap);
-          if constexpr (!ADJ) {
-            acc0 = fmaf(Gf, ec, acc0);
-            acc1 = fmaf(Gf, s_own, acc1);
-            if (mrow) {
-#pragma unroll
-              for (int bb = 0; bb < BT; ++bb) mrow[tm.state(u, jj, bb)] = e[bb] * Gf;
-            }
-          } else {
-            const float base = fa[u][jj] - Dc;
-#pragma unroll
-            for (int bb = 0; bb < BT; ++bb) {
-              const float gam = e[bb] * Gf;
-              const float psi = gam * (base + eps[bb]);
-              acc0 = fmaf(psi, cb[u][jj][bb], acc0);
-              if (active)
-                gc[u][jj][bb] += fmaf(gt, gam, psi * fmaf(-p.two_over_T, cb[u][jj][bb], tw));
-            }
-          }
-        }
-      }
-      // Per-step partial sums, one pair per warp (per team when narrower).
-      {
-        const float v0 = group_sum(acc0, tm.width);
-        const float v1 = ADJ ? 0.f : group_sum(acc1, tm.width);
-        if ((tm.lane & (tm.width - 1)) == 0) {
-          part[(static_cast<size_t>(t) * 2 + 0) * tm.wpt + tm.warp_in_team] = v0;
-          if constexpr (!ADJ) part[(static_cast<size_t>(t) * 2 + 1) * tm.wpt + tm.warp_in_team] = v1;
-        }
-      }
-      if (t >= 1) {
-        float lmax = kNegInf;
-        if (tm.b_writer) {
-#pragma unroll
-          for (int u = 0; u < U; ++u)
-#pragma unroll
-            for (int jj = 0; jj < JT; ++jj) {
-              lmax = fmaxf(lmax, bo[u][jj]);
-              uint32_t r;
-              int off;
-              tm.b_dest(tm.b_out_index(u, jj), r, off);
-              team_store<CL>(bufB + ((t - 1) & 1) * GL, r, off, bo[u][jj]);
-              if constexpr (ADJ) team_store<CL>(bufBt + ((t - 1) & 1) * GL, r, off, bto[u][jj]);
-            }
-        }
-        const float wm = publish_max(tm, maxp + ((t - 1) & 1) * 128, lmax);
-        team_sync<CL>();
-        const float Mn = collect_max(tm, maxp + ((t - 1) & 1) * 128, wm);
-        Dt += static_cast<double>(Mb);
-        Mb = Mn;
-      }
-    }
-    team_sync<CL>();
-    // Per-step outputs from the partial sums (fixed order: deterministic).
-    if (active) {
-      for (int t = tm.tt; t < n; t += tm.TS) {
-        float v0 = 0.f, v1 = 0.f;
-        for (int i = 0; i < tm.wpt; ++i) {
-          v0 += part[(static_cast<size_t>(t) * 2 + 0) * tm.wpt + i];
-          if constexpr (!ADJ) v1 += part[(static_cast<size_t>(t) * 2 + 1) * tm.wpt + i];
-        }
-        if constexpr (!ADJ) {
-          p.w_hat[static_cast<size_t>(seq) * n + t] = v0 / v1;
-        } else {
-          p.grad_w[static_cast<size_t>(seq) * n + t] = p.two_over_T * v0;
-        }
-      }
-    }
-    team_sync<CL>();
-  }
-
-  if constexpr (ADJ) {
-    float* gp = p.gc_part + static_cast<size_t>(slot) * S;
-#pragma unroll
-    for (int u = 0; u < U; ++u)
-#pragma unroll
-      for (int jj = 0; jj < JT; ++jj)
-#pragma unroll
-        for (int bb = 0; bb < BT; ++bb) gp[tm.state(u, jj, bb)] = gc[u][jj][bb];
-  }
-  if constexpr (CL > 1) cluster_sync_all();  // no CTA leaves while its shared memory may be addressed
-}
 
 // ---------------------------------------------------------------------------
 // Hard decode: max-sum over -(w - c)^2 in float64, each difference, square and
@@ -604,6 +55,9 @@ __global__ void __launch_bounds__(NTB, 1) viterbi_kernel(const ViterbiParams p) 
       for (int bb = 0; bb < BT; ++bb) cb[u][jj][bb] = __ldg(p.codebook + tm.state(u, jj, bb));
 
   uint8_t* bp = p.bp + static_cast<size_t>(slot) * p.bp_stride;
+  // Every CTA of the cluster must be running before any of them writes into
+  // another's shared memory.
+  if constexpr (CL > 1) cluster_sync_all();
   const int iters = (p.N + p.num_slots - 1) / p.num_slots;
   for (int it = 0; it < iters; ++it) {
     const int seq_raw = slot + it * p.num_slots;
@@ -742,22 +196,24 @@ __global__ void gradc_reduce_kernel(const float* __restrict__ part, int num_slot
 // ---------------------------------------------------------------------------
 // Host side: geometry and launches.
 // ---------------------------------------------------------------------------
+const void* fb_fwd_kernel_k1(int cluster, int nseq);
+const void* fb_fwd_kernel_k2(int cluster, int nseq);
+const void* fb_fwd_kernel_k3(int cluster, int nseq);
+const void* fb_fwd_kernel_k4(int cluster, int nseq);
+const void* fb_adj_kernel_k1(int cluster, int nseq);
+const void* fb_adj_kernel_k2(int cluster, int nseq);
+const void* fb_adj_kernel_k3(int cluster, int nseq);
+const void* fb_adj_kernel_k4(int cluster, int nseq);
+
 namespace {
 
-template <int K, int CL, bool ADJ, int NTB>
-const void* fb_fn() {
-  return reinterpret_cast<const void*>(&fb_kernel<K, CL, ADJ, NTB>);
-}
-
-template <bool ADJ>
-const void* pick_fb(int k, int cl) {
-#define BCJR_FB_CASE(KK, CC)                                  \
-  if (k == KK && cl == CC) return fb_fn<(1 << KK), CC, ADJ, 1024>();
-  BCJR_FB_CASE(1, 1) BCJR_FB_CASE(1, 2) BCJR_FB_CASE(1, 4)
-  BCJR_FB_CASE(2, 1) BCJR_FB_CASE(2, 2) BCJR_FB_CASE(2, 4)
-  BCJR_FB_CASE(3, 1) BCJR_FB_CASE(3, 2) BCJR_FB_CASE(3, 4)
-  BCJR_FB_CASE(4, 1) BCJR_FB_CASE(4, 2) BCJR_FB_CASE(4, 4)
-#undef BCJR_FB_CASE
+const void* pick_fb(bool adjoint, int k, int cl, int nseq) {
+  switch (k) {
+    case 1: return adjoint ? fb_adj_kernel_k1(cl, nseq) : fb_fwd_kernel_k1(cl, nseq);
+    case 2: return adjoint ? fb_adj_kernel_k2(cl, nseq) : fb_fwd_kernel_k2(cl, nseq);
+    case 3: return adjoint ? fb_adj_kernel_k3(cl, nseq) : fb_fwd_kernel_k3(cl, nseq);
+    case 4: return adjoint ? fb_adj_kernel_k4(cl, nseq) : fb_fwd_kernel_k4(cl, nseq);
+  }
   return nullptr;
 }
 
@@ -772,12 +228,13 @@ const void* pick_viterbi(int k, int cl) {
   return nullptr;
 }
 
-void base_geometry(int L, TeamGeometry* g) {
+// Team shape for a given maximum CTA size.
+void base_geometry(int L, int max_block, TeamGeometry* g) {
   const int TS = (1 << L) / kStatesPerThread;
   g->team_threads = TS;
-  if (TS > 1024) {
-    g->block_threads = 1024;
-    g->cluster = TS / 1024;
+  if (TS > max_block) {
+    g->block_threads = max_block;
+    g->cluster = TS / max_block;
     g->teams_per_cta = 1;
   } else if (TS >= 32) {
     g->block_threads = TS;
@@ -789,17 +246,26 @@ void base_geometry(int L, TeamGeometry* g) {
     g->teams_per_cta = 32 / TS;
   }
   g->warps_per_team = TS < 32 ? 1 : TS / 32;
+  g->nseq = 1;
 }
 
-cudaError_t persistent_grid(const void* fn, int n_seq, TeamGeometry* g) {
-  int dev0 = 0, max_smem = 0;
-  cudaError_t e = cudaGetDevice(&dev0);
-  if (e != cudaSuccess) return e;
-  if ((e = cudaDeviceGetAttribute(&max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev0)) != cudaSuccess)
-    return e;
-  if (g->smem_bytes > static_cast<size_t>(max_smem)) return cudaErrorNotSupported;
-  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(g->smem_bytes));
+int max_optin_smem() {
+  int dev = 0, v = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return 0;
+  return v;
+}
+
+// Persistent grid: as many teams as can be resident, no more than there is work for.
+// One kernel function serves several team sizes, so its dynamic shared-memory
+// limit is raised once to the device maximum rather than to one launch's need.
+cudaError_t allow_max_smem(const void* fn) {
+  return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, max_optin_smem());
+}
+
+cudaError_t persistent_grid(const void* fn, int work_units, TeamGeometry* g) {
+  if (g->smem_bytes > static_cast<size_t>(max_optin_smem())) return cudaErrorNotSupported;
+  cudaError_t e = allow_max_smem(fn);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
@@ -827,8 +293,8 @@ cudaError_t persistent_grid(const void* fn, int n_seq, TeamGeometry* g) {
       return e;
     resident_teams = per_sm * sms * g->teams_per_cta;
   }
-  if (resident_teams < 1) return cudaErrorInvalidConfiguration;
-  int slots = n_seq < resident_teams ? n_seq : resident_teams;
+  if (resident_teams < 1) return cudaErrorNotSupported;
+  int slots = work_units < resident_teams ? work_units : resident_teams;
   if (slots < 1) slots = 1;
   if (g->cluster > 1) {
     g->num_slots = slots;
@@ -857,30 +323,95 @@ cudaError_t launch(const void* fn, const TeamGeometry& g, void** args, cudaStrea
   return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
+int states_per_thread_values(int k) {  // floats per thread in a thread-private row
+  const int K = 1 << k;
+  const int JT = K < 4 ? K : 4;
+  const int U = K <= 4 ? 16 / (K * K) : 1;
+  return U * JT;
+}
+
 }  // namespace
 
-cudaError_t fb_geometry(int L, int k, int n_seq, bool adjoint, TeamGeometry* g) {
-  base_geometry(L, g);
+namespace {
+
+// Geometry depends only on (device, sizes); computing it queries occupancy,
+// so it is cached per process.
+using GeoKey = std::tuple<int, int, int, int, int, int, int>;
+std::mutex g_geo_mu;
+std::map<GeoKey, std::pair<cudaError_t, TeamGeometry>> g_geo_cache;
+
+cudaError_t fb_geometry_uncached(int L, int k, int n_seq, bool adjoint, int C, int nseq_request, TeamGeometry* g) {
+  base_geometry(L, adjoint ? 512 : 1024, g);
   const int GL = ((1 << L) >> k) / g->cluster;
-  const size_t per_team = adjoint ? fb_smem_floats_per_team<true>(GL) : fb_smem_floats_per_team<false>(GL);
-  g->smem_bytes = per_team * sizeof(float) * g->teams_per_cta;
-  const void* fn = adjoint ? pick_fb<true>(k, g->cluster) : pick_fb<false>(k, g->cluster);
-  if (!fn) return cudaErrorInvalidValue;
-  return persistent_grid(fn, n_seq, g);
+  const int NV = states_per_thread_values(k);
+  const bool alias = (C == 1);
+  const int max_smem = max_optin_smem();
+  (void)nseq_request;
+  const int nseq = 1;  // one sequence in flight per team
+  const size_t smem = fb_smem_layout(GL, g->block_threads, NV, nseq, adjoint, alias, g->teams_per_cta).total;
+  if (smem > static_cast<size_t>(max_smem)) return cudaErrorNotSupported;
+  g->nseq = nseq;
+  g->smem_bytes = smem;
+  const void* fn = pick_fb(adjoint, k, g->cluster, nseq);
+  if (!fn) return cudaErrorNotSupported;
+  return persistent_grid(fn, (n_seq + nseq - 1) / nseq, g);
+}
+
+}  // namespace
+
+cudaError_t fb_geometry(int L, int k, int n_seq, bool adjoint, int C, int nseq_request, TeamGeometry* g) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const GeoKey key{dev, L, k, n_seq, adjoint ? 1 : 0, C == 1 ? 1 : 0, nseq_request == 1 ? 3 : 0};
+  {
+    std::lock_guard<std::mutex> lk(g_geo_mu);
+    auto it = g_geo_cache.find(key);
+    if (it != g_geo_cache.end()) {
+      *g = it->second.second;
+      return it->second.first;
+    }
+  }
+  TeamGeometry gg = {};
+  e = fb_geometry_uncached(L, k, n_seq, adjoint, C, nseq_request, &gg);
+  if (e == cudaSuccess || e == cudaErrorNotSupported) {
+    std::lock_guard<std::mutex> lk(g_geo_mu);
+    g_geo_cache[key] = {e, gg};
+  }
+  *g = gg;
+  return e;
 }
 
 cudaError_t viterbi_geometry(int L, int k, int n_seq, TeamGeometry* g) {
-  base_geometry(L, g);
-  const int GL = ((1 << L) >> k) / g->cluster;
-  g->smem_bytes = (2 * static_cast<size_t>(GL) + 2 * 128) * sizeof(double) * g->teams_per_cta;
-  const void* fn = pick_viterbi(k, g->cluster);
-  if (!fn) return cudaErrorInvalidValue;
-  return persistent_grid(fn, n_seq, g);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const GeoKey key{dev, L, k, n_seq, 2, 0, 1};
+  {
+    std::lock_guard<std::mutex> lk(g_geo_mu);
+    auto it = g_geo_cache.find(key);
+    if (it != g_geo_cache.end()) {
+      *g = it->second.second;
+      return it->second.first;
+    }
+  }
+  TeamGeometry gg = {};
+  base_geometry(L, 1024, &gg);
+  const int GL = ((1 << L) >> k) / gg.cluster;
+  gg.smem_bytes = (2 * static_cast<size_t>(GL) + 2 * 128) * sizeof(double) * gg.teams_per_cta;
+  const void* fn = pick_viterbi(k, gg.cluster);
+  e = fn ? persistent_grid(fn, n_seq, &gg) : cudaErrorNotSupported;
+  if (e == cudaSuccess || e == cudaErrorNotSupported) {
+    std::lock_guard<std::mutex> lk(g_geo_mu);
+    g_geo_cache[key] = {e, gg};
+  }
+  *g = gg;
+  return e;
 }
 
 cudaError_t launch_fb(const FBParams& p, const TeamGeometry& g, bool adjoint, cudaStream_t s) {
-  const void* fn = adjoint ? pick_fb<true>(p.k, g.cluster) : pick_fb<false>(p.k, g.cluster);
-  if (!fn) return cudaErrorInvalidValue;
+  const void* fn = pick_fb(adjoint, p.k, g.cluster, g.nseq);
+  if (!fn) return cudaErrorNotSupported;
   FBParams copy = p;
   void* args[] = {&copy};
   return launch(fn, g, args, s);
@@ -888,7 +419,7 @@ cudaError_t launch_fb(const FBParams& p, const TeamGeometry& g, bool adjoint, cu
 
 cudaError_t launch_viterbi(const ViterbiParams& p, const TeamGeometry& g, cudaStream_t s) {
   const void* fn = pick_viterbi(p.k, g.cluster);
-  if (!fn) return cudaErrorInvalidValue;
+  if (!fn) return cudaErrorNotSupported;
   ViterbiParams copy = p;
   void* args[] = {&copy};
   return launch(fn, g, args, s);

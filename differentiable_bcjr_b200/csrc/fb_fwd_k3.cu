@@ -1,0 +1,13 @@
+// fb_fwd_k3.cu -- instantiations of the fused forward-backward kernel, k = 3 (soft codeword).
+#include "fb_kernel.cuh"
+
+namespace bcjr {
+
+const void* fb_fwd_kernel_k3(int cluster, int nseq) {
+  if (cluster == 1 && nseq == 1) return reinterpret_cast<const void*>(&fb_kernel<8, 1, false, 1, 1024>);
+  if (cluster == 2 && nseq == 1) return reinterpret_cast<const void*>(&fb_kernel<8, 2, false, 1, 1024>);
+  if (cluster == 4 && nseq == 1) return reinterpret_cast<const void*>(&fb_kernel<8, 4, false, 1, 1024>);
+  return nullptr;
+}
+
+}  // namespace bcjr

@@ -1,0 +1,13 @@
+// fb_fwd_k4.cu -- instantiations of the fused forward-backward kernel, k = 4 (soft codeword).
+#include "fb_kernel.cuh"
+
+namespace bcjr {
+
+const void* fb_fwd_kernel_k4(int cluster, int nseq) {
+  if (cluster == 1 && nseq == 1) return reinterpret_cast<const void*>(&fb_kernel<16, 1, false, 1, 1024>);
+  if (cluster == 2 && nseq == 1) return reinterpret_cast<const void*>(&fb_kernel<16, 2, false, 1, 1024>);
+  if (cluster == 4 && nseq == 1) return reinterpret_cast<const void*>(&fb_kernel<16, 4, false, 1, 1024>);
+  return nullptr;
+}
+
+}  // namespace bcjr

@@ -59,7 +59,10 @@ typedef struct {
   /* Keep the forward group vector every C steps and recompute the others
    * during the backward sweep; 0 selects C = 1 (keep every step). */
   int checkpoint_interval;
-  int reserved[7]; /* set to zero */
+  /* Sequences a thread-block cluster keeps in flight: 0 = automatic, 1.
+   * (Other values are rejected; the interleaved schedule is not offered.) */
+  int sequences_in_flight;
+  int reserved[6]; /* set to zero */
 } bcjr_options;
 
 typedef enum {

@@ -84,8 +84,13 @@ def test_checkpoint_interval_gives_the_same_answer(B, L, k, n, N, T, C):
     assert_abs(w_hat, o_what, W_HAT_ATOL, "w_hat")
     assert_rel_l2(grad_w, o_gw, GRAD_REL_L2, "grad_w")
     assert_rel_l2(grad_c, o_gc, GRAD_REL_L2, "grad_codebook")
-    # recomputation repeats the stored steps bit for bit
-    assert torch.equal(w_hat, w_hat1) and torch.equal(grad_w, grad_w1) and torch.equal(grad_c, grad_c1)
+    # C > 1 runs another kernel instantiation (one sequence in flight per team,
+    # the forward values recomputed per segment); the per-sequence outputs agree
+    # to a few ulp, and grad_codebook sums the sequences in another order
+    torch.testing.assert_close(log_z, log_z1, rtol=1e-6, atol=1e-6)
+    torch.testing.assert_close(w_hat, w_hat1, rtol=0, atol=1e-6)
+    torch.testing.assert_close(grad_w, grad_w1, rtol=1e-5, atol=1e-5)
+    torch.testing.assert_close(grad_c, grad_c1, rtol=1e-5, atol=1e-5)
 
 
 @pytest.mark.parametrize("L,k,n,N", [(8, 2, 64, 16), (4, 1, 7, 5), (6, 3, 9, 4), (9, 2, 12, 3), (12, 4, 10, 3),
@@ -96,6 +101,15 @@ def test_viterbi_bit_exact(B, L, k, n, N):
     o_states, o_hard, _ = oracle.viterbi(w, c, L, k)
     np.testing.assert_array_equal(states.cpu().numpy(), o_states)
     np.testing.assert_array_equal(w_hard.cpu().numpy(), o_hard)
+
+
+def test_alternating_sizes_share_kernels(B):
+    # L = 10 and L = 9 (k = 3) use the same kernel instantiation with different
+    # shared-memory sizes; going back to the larger one must still launch.
+    for L in (10, 9, 10, 9):
+        (c, w, g), (w_hat, _, _, grad_w, _) = _run_fwd_bwd(B, L, 3, 6, 2, 0.4, seed=L)
+        o_what, _, _ = oracle.forward(w, c, 0.4, L, 3)
+        assert_abs(w_hat, o_what, W_HAT_ATOL, f"w_hat L={L}")
 
 
 def test_single_step_and_empty_batch(B):
