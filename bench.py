@@ -20,8 +20,10 @@ a bounded sample of the same workload (whole sequences), same metric.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -44,7 +46,7 @@ ALG_MUFU_PER_STATE_STEP = 4       # one forward and one backward log-sum-exp in 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=8)
+    ap.add_argument("--steps", type=int, default=4)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -193,13 +195,27 @@ def load_peaks():
         return {}
 
 
+def kernel_source_hash():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "differentiable_bcjr_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(f.encode())
+            h.update(open(os.path.join(d, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
 def load_traffic():
-    """dram bytes per launch of the dominant kernel from the committed ncu summary, if current."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    """DRAM bytes per launch from the committed ncu summary, or {} once the kernels changed."""
+    p = os.path.join(ROOT, "profiles", "fb_kernel_L16_k2_full.md")
     try:
-        return json.load(open(p))
-    except Exception:
+        text = open(p).read()
+    except OSError:
         return {}
+    m = re.search(r"^kernel_source_sha256_16: (\w+)", text, re.M)
+    if not m or m.group(1) != kernel_source_hash():
+        return {}
+    return {k: int(v) for k, v in re.findall(r"^(\w+_dram_bytes_per_launch): (\d+)", text, re.M)}
 
 
 def run_gpu(args):
