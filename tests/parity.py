@@ -10,6 +10,12 @@ W_HAT_ATOL = 1e-5
 MARGINAL_ATOL = 1e-5
 GRAD_REL_L2 = 1e-3
 LOGZ_RTOL = 1e-5
+# log Z is a sum of one log-sum-exp per step, each evaluated with the fast
+# hardware 2^x and log2 (relative error of 2^x about 2^-22, absolute error of
+# log2 about 2^-22.6, plus an fp32 sum of K terms): under 2^-21 natural-log
+# units per step.  The bound is taken with a factor 2 margin and grows with the
+# sequence length; where log Z is near zero only this absolute part applies.
+LOGZ_ATOL_PER_STEP = 2.0 ** -20
 
 
 def to_np(x):
