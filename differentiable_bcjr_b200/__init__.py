@@ -53,6 +53,7 @@ _Z = ctypes.c_size_t
 _SIGS = {
     "bcjr_workspace_size": (_Z, [_I, _I, _I, _I, _I, ctypes.POINTER(Options)]),
     "bcjr_forward": (_I, [_P, _P, _F, _I, _I, _I, _I, _P, _P, _P, ctypes.POINTER(Options), _P, _Z, _P]),
+    "bcjr_forward_static_scratch": (_I, [_P, _P, _F, _I, _I, _I, _I, _P, _P, _P, ctypes.POINTER(Options), _P]),
     "bcjr_backward": (_I, [_P, _P, _P, _P, _F, _I, _I, _I, _I, _P, _P, _I, ctypes.POINTER(Options), _P, _Z,
                            _P]),
     "viterbi_decode": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _Z, _P]),
@@ -163,6 +164,23 @@ def bcjr_forward(w, codebook, T, state_bits, k, want_marginals=False, checkpoint
                               _ptr(log_z), ctypes.byref(o), _ptr(wsb), wsb.numel(), _stream(dev)),
            "bcjr_forward")
     return w_hat, marg, log_z
+
+
+STATIC_SCRATCH_BYTES = 32 << 20
+
+
+def bcjr_forward_static_scratch(w, codebook, T, state_bits, k, w_hat, log_z=None, marginals=None,
+                                checkpoint_interval=0):
+    """bcjr_forward into caller-provided outputs, with the library's static
+    device scratch as workspace: neither this function nor the library
+    allocates device memory.  Calls on one device share that scratch, so they
+    must not overlap in time."""
+    _need_cuda(w, codebook, w_hat, log_z, marginals)
+    N, n = w.shape
+    o = _opts(checkpoint_interval)
+    _check(lib().bcjr_forward_static_scratch(_ptr(w), _ptr(codebook), float(T), state_bits, k, n, N, _ptr(w_hat),
+                                             _ptr(marginals), _ptr(log_z), ctypes.byref(o), _stream(w.device)),
+           "bcjr_forward_static_scratch")
 
 
 def bcjr_backward(grad_w_hat, w, codebook, w_hat, T, state_bits, k, checkpoint_interval=0, ws=None,

@@ -95,6 +95,32 @@ bcjr_status bcjr_forward(const float* w, const float* codebook, float T, int sta
                          bcjr_stream_t stream);
 
 /*
+ * bcjr_forward without a workspace argument: the same computation and outputs,
+ * with scratch taken from a statically allocated device array of
+ * BCJR_STATIC_SCRATCH_BYTES per device, so the call allocates no memory and
+ * needs none from the caller.  The paper has no counterpart; this is a library
+ * convenience for callers that cannot allocate device memory at call time.
+ *  - The first call on each device looks up that device's copy of the array
+ *    (which may load the library's module on it) and sets up the launch
+ *    geometry; make that first call before any stream capture.  No claim is
+ *    made about use inside a CUDA graph capture.
+ *  - Returns BCJR_ERR_WORKSPACE, before launching anything, when the problem
+ *    needs more than BCJR_STATIC_SCRATCH_BYTES, i.e. when
+ *    bcjr_workspace_size(BCJR_OP_FORWARD, ...) is larger.
+ *  - The device-side status word lives in the array and is cleared at the
+ *    start of every call; a non-finite log-partition function shows as a
+ *    non-finite log_z (bcjr_get_status cannot reach this scratch).
+ *  - All calls on one device share the one array: two calls whose work
+ *    overlaps in time (on different streams, or from several host threads
+ *    without ordering) race on it and give wrong results.  Order them on one
+ *    stream or with events.
+ */
+#define BCJR_STATIC_SCRATCH_BYTES (32u << 20) /* 32 MiB */
+bcjr_status bcjr_forward_static_scratch(const float* w, const float* codebook, float T, int state_bits,
+                                        int k, int seq_len, int n_seq, float* w_hat, float* marginals,
+                                        float* log_z, const bcjr_options* opt, bcjr_stream_t stream);
+
+/*
  * Vector-Jacobian product of the soft codeword ("key technical innovations":
  * exact gradients through the trellis, differentiable in the weight preimage
  * and the trellis parameters).  With L = sum_t grad_w_hat_t w_hat_t:
