@@ -196,10 +196,11 @@ def load_peaks():
 
 
 def kernel_source_hash():
+    """Hash of the sources that define the forward-backward kernels."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "differentiable_bcjr_b200", "csrc")
     for f in sorted(os.listdir(d)):
-        if f.endswith((".cu", ".cuh", ".h")):
+        if f.startswith(("fb_", "bcjr_device", "team", "bcjr_internal")):
             h.update(f.encode())
             h.update(open(os.path.join(d, f), "rb").read())
     return h.hexdigest()[:16]
