@@ -41,8 +41,8 @@ int effective_c(const bcjr_options* opt, int n) {
 // Byte offsets of every workspace region for one bitshift call.  "Lanes" are
 // the sequences in flight: teams x sequences per team.
 struct FBLayout {
-  size_t ck, ckF, ck64, ckF64, Mtab, Ctab, part, gc, total;
-  size_t ck_stride, ck64_stride, tab_stride, part_stride, row;
+  size_t ck, ckR, ckF, ck64, ckF64, part, gc, total;
+  size_t ck_stride, ckR_stride, ck64_stride, part_stride, row;
 };
 
 // Elements of one thread-private checkpoint row: (S/16 threads) x (forward
@@ -57,25 +57,25 @@ size_t ckpt_row(int L, int k) {
 FBLayout fb_layout(const TeamGeometry& g, int L, int k, int n, int C, bool adjoint) {
   FBLayout l = {};
   const size_t row = ckpt_row(L, k);
+  const size_t team_threads = (static_cast<size_t>(1) << L) / 16;
   const size_t lanes = static_cast<size_t>(g.num_slots) * g.nseq;
+  const size_t rows = C == 1 ? static_cast<size_t>(n) : static_cast<size_t>(C);
   l.row = row;
-  l.ck_stride = (C == 1 ? static_cast<size_t>(n) : static_cast<size_t>(C)) * row;
+  l.ck_stride = rows * row;
+  l.ckR_stride = rows * team_threads;
   l.ck64_stride = C == 1 ? 0 : static_cast<size_t>((n - 1) / C + 1) * row;
-  l.tab_stride = static_cast<size_t>(n) + 1;
   l.part_stride = static_cast<size_t>(n) * 2 * g.warps_per_team;
   size_t off = kHeaderBytes;
   l.ck = off;
   off = align_up(off + lanes * l.ck_stride * sizeof(float));
+  l.ckR = off;
+  off = align_up(off + lanes * l.ckR_stride * sizeof(uint32_t));
   l.ckF = off;
   if (adjoint) off = align_up(off + lanes * l.ck_stride * sizeof(float));
   l.ck64 = off;
   off = align_up(off + lanes * l.ck64_stride * sizeof(double));
   l.ckF64 = off;
   if (adjoint) off = align_up(off + lanes * l.ck64_stride * sizeof(float));
-  l.Mtab = off;
-  off = align_up(off + lanes * l.tab_stride * sizeof(float));
-  l.Ctab = off;
-  off = align_up(off + lanes * l.tab_stride * sizeof(double));
   l.part = off;
   off = align_up(off + lanes * l.part_stride * sizeof(float));
   l.gc = off;
@@ -191,19 +191,18 @@ static bcjr_status fb_common(bool adjoint, const float* grad_w_hat, const float*
   p.grad_w = grad_w;
   p.gc_part = reinterpret_cast<float*>(base + lay.gc);
   p.ck = reinterpret_cast<float*>(base + lay.ck);
+  p.ckR = reinterpret_cast<uint32_t*>(base + lay.ckR);
   p.ckF = reinterpret_cast<float*>(base + lay.ckF);
   p.ck64 = reinterpret_cast<double*>(base + lay.ck64);
   p.ckF64 = reinterpret_cast<float*>(base + lay.ckF64);
-  p.Mtab = reinterpret_cast<float*>(base + lay.Mtab);
-  p.Ctab = reinterpret_cast<double*>(base + lay.Ctab);
   p.part = reinterpret_cast<float*>(base + lay.part);
   p.status = reinterpret_cast<int*>(base);
   p.ck_stride = lay.ck_stride;
+  p.ckR_stride = lay.ckR_stride;
   p.ck64_stride = lay.ck64_stride;
-  p.tab_stride = lay.tab_stride;
   p.part_stride = lay.part_stride;
   p.row = lay.row;
-  p.sc64 = 1.4426950408889634 / static_cast<double>(T);
+  p.sqsc = std::sqrt(1.4426950408889634 / static_cast<double>(T));
   p.two_over_T = static_cast<float>(2.0 / static_cast<double>(T));
   p.L = L;
   p.k = k;

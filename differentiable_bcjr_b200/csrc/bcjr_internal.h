@@ -39,20 +39,19 @@ struct FBParams {
   // thread tt of the team owns elements [tt*NV, tt*NV + NV) of every row, so a
   // row holds team_threads * NV values (= S/2^k for k <= 2, S/4 for k >= 3,
   // where lanes sharing a forward group each keep their own copy).
-  float* ck;               // C == 1: [n][row] forward values A_t - M_t (float); C > 1: ring [C][row]
-  float* ckF;              // same for the forward adjoint accumulators (backward)
-  double* ck64;            // C > 1: [n/C + 1][row] A_t - M_t at t = 0, C, 2C, ... (float64)
+  float* ck;               // C == 1: [n][row] forward values A'_t - R - 1 (float); C > 1: ring [C][row]
+  uint32_t* ckR;           // C == 1: [n][team_threads] high word of each thread's reference R; C > 1: ring [C][...]
+  float* ckF;              // same layout as ck for the forward adjoint accumulators (backward)
+  double* ck64;            // C > 1: [n/C + 1][row] A'_t at t = 0, C, 2C, ... (float64)
   float* ckF64;            // C > 1: [n/C + 1][row] forward adjoint accumulators at the same t
-  float* Mtab;             // [n + 1] team max M_t of the raw forward vector
-  double* Ctab;            // [n + 1] log2 scale C_{t+1} = C_t + M_t of the forward vector
   float* part;             // [n][2][warps_per_team] per-warp partial sums
   int* status;
   size_t ck_stride;        // floats per lane in ck / ckF
+  size_t ckR_stride;       // words per lane in ckR
   size_t ck64_stride;      // elements per lane in ck64 / ckF64
-  size_t tab_stride;       // entries per lane in Mtab / Ctab
   size_t part_stride;      // floats per lane in part
   size_t row;              // elements per checkpoint row (team_threads * NV)
-  double sc64;             // log2(e) / T
+  double sqsc;             // sqrt(log2(e) / T): emission phi = -((w - c) sqsc)^2 in log2 units
   float two_over_T;
   int L, k, n, N, C;
   int num_slots;
@@ -60,11 +59,11 @@ struct FBParams {
 
 // Shared-memory carve-up of the forward-backward kernel (bytes), identical on
 // host and device.  Per team and per sequence in flight: the double-buffered
-// exchange vectors (float64 group values, float32 adjoint accumulators) and
-// the per-warp maxima; per CTA: a reduction scratch and the thread-private
-// staging of the forward values read by the backward sweep.
+// exchange vectors (float64 group values, float32 adjoint accumulators); per
+// CTA: a reduction scratch and the thread-private staging of the forward
+// values read by the backward sweep (values, reference words, accumulators).
 struct FBSmem {
-  uint32_t exA, exF, exB, exBt, maxp, per_seq, per_team, red, stage, stageF, total;
+  uint32_t exA, exF, exB, exBt, per_seq, per_team, red, stage, stageK, stageF, total;
 };
 __host__ __device__ inline FBSmem fb_smem_layout(int GL, int NT, int NV, int nseq, bool adj, bool alias,
                                                  int teams_per_cta) {
@@ -78,16 +77,19 @@ __host__ __device__ inline FBSmem fb_smem_layout(int GL, int NT, int NV, int nse
   if (!alias) o += 2u * GL * 8u;
   l.exBt = alias ? l.exF : o;
   if (!alias && adj) o += 2u * GL * 4u;
-  l.maxp = o;
-  o += 2u * 128u * 4u;
+  o = (o + 15u) & ~15u;
   l.per_seq = o;
   l.per_team = static_cast<uint32_t>(nseq) * o;
   l.red = static_cast<uint32_t>(teams_per_cta) * l.per_team;
   o = l.red + 4u * 128u * 4u;
+  // staging of the stored forward values (C == 1 only; C > 1 reads its ring directly)
+  const uint32_t stg = alias ? static_cast<uint32_t>(nseq) * 2u * NT : 0u;
   l.stage = o;
-  o += static_cast<uint32_t>(nseq) * 2u * NT * NV * 4u;
+  o += stg * NV * 4u;
   l.stageF = o;
-  if (adj) o += static_cast<uint32_t>(nseq) * 2u * NT * NV * 4u;
+  if (adj) o += stg * NV * 4u;
+  l.stageK = o;
+  o += stg * 4u;
   l.total = o;
   return l;
 }

@@ -207,6 +207,8 @@ const void* fb_adj_kernel_k4(int cluster, int nseq);
 
 namespace {
 
+constexpr int kFBBlockThreads = 512;  // 16 states per thread, <= 128 registers per thread
+
 const void* pick_fb(bool adjoint, int k, int cl, int nseq) {
   switch (k) {
     case 1: return adjoint ? fb_adj_kernel_k1(cl, nseq) : fb_fwd_kernel_k1(cl, nseq);
@@ -341,13 +343,15 @@ std::mutex g_geo_mu;
 std::map<GeoKey, std::pair<cudaError_t, TeamGeometry>> g_geo_cache;
 
 cudaError_t fb_geometry_uncached(int L, int k, int n_seq, bool adjoint, int C, int nseq_request, TeamGeometry* g) {
-  base_geometry(L, adjoint ? 512 : 1024, g);
+  base_geometry(L, kFBBlockThreads, g);
   const int GL = ((1 << L) >> k) / g->cluster;
   const int NV = states_per_thread_values(k);
   const bool alias = (C == 1);
   const int max_smem = max_optin_smem();
   (void)nseq_request;
-  const int nseq = 1;  // one sequence in flight per team
+  // Clusters keep two sequences in flight (the barrier of one hides behind the
+  // other's step); k = 1 has twice the group values and keeps one.
+  const int nseq = (g->cluster > 1 && k >= 2) ? 2 : 1;
   const size_t smem = fb_smem_layout(GL, g->block_threads, NV, nseq, adjoint, alias, g->teams_per_cta).total;
   if (smem > static_cast<size_t>(max_smem)) return cudaErrorNotSupported;
   g->nseq = nseq;

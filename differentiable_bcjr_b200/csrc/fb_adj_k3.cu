@@ -5,9 +5,9 @@ namespace bcjr {
 
 const void* fb_adj_kernel_k3(int cluster, int nseq) {
   if (cluster == 1 && nseq == 1) return reinterpret_cast<const void*>(&fb_kernel<8, 1, true, 1, 512>);
-  if (cluster == 2 && nseq == 1) return reinterpret_cast<const void*>(&fb_kernel<8, 2, true, 1, 512>);
-  if (cluster == 4 && nseq == 1) return reinterpret_cast<const void*>(&fb_kernel<8, 4, true, 1, 512>);
-  if (cluster == 8 && nseq == 1) return reinterpret_cast<const void*>(&fb_kernel<8, 8, true, 1, 512>);
+  if (cluster == 2 && nseq == 2) return reinterpret_cast<const void*>(&fb_kernel<8, 2, true, 2, 512>);
+  if (cluster == 4 && nseq == 2) return reinterpret_cast<const void*>(&fb_kernel<8, 4, true, 2, 512>);
+  if (cluster == 8 && nseq == 2) return reinterpret_cast<const void*>(&fb_kernel<8, 8, true, 2, 512>);
   return nullptr;
 }
 

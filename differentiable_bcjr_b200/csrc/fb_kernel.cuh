@@ -10,32 +10,43 @@
 // Trellis: pred(s) = {(j << (L-k)) | (s >> k) : j < K}, K = 2^k; emission
 // log-weight phi_t(s) = -(w_t - c(s))^2 / T; uniform start; free end.
 //
-// Group form (an exact rewrite of the forward-backward):
+// Group form (an exact rewrite of the forward-backward), in base 2:
 //   alpha_t(s) = phi_t(s) + A_t(s >> k),  A_{t+1}(g) = LSE_j alpha_t((j << (L-k)) | g)
 //   beta_t(p)  = B_t(p & (S/K-1)),        B_{t-1}(h) = LSE_b [phi_t((h << k) | b) + B_t(((h << k) | b) & (S/K-1))]
-// A sweep step is one K-term log-sum-exp per group of K states; only S/K
+// A sweep step is one K-term log-sum-exp per group of K states; only the S/K
 // group values move between threads.
 //
-// Arithmetic.  Base 2 throughout.  The emission and the running group values
-// are float64 (the log-domain values of competing paths differ by tens of
-// units at T = 0.005, where float32 rounding would accumulate along a path);
-// exponentials and logarithms are the float32 MUFU ex2/lg2 of differences that
-// are small for every term that matters.  Every step subtracts the exact
-// team-wide maximum M_t of the incoming vector; the shifts are summed in
-// float64 (C_t forward, D_t backward).  The backward log-sum-exp is referenced
-// to the posterior itself: its terms are gamma_t(s) = 2^{y_b + r_h}, with
-// r_h = A_t(h) - M_t + C_{t+1} + M'_t + D_t - log2 Z, so one exponential per
-// state yields both the marginal and the backward recursion.
+// Arithmetic.
+//  * Emission: with c'(s) = c(s) sqrt(log2(e)/T) and w'_t likewise,
+//    phi_t(s) = -(w'_t - c'(s))^2 in log2 units: one float64 subtract and one
+//    float64 fma per state (c' stays in registers as float64).
+//  * Running values are float64 and carry a fixed drift instead of a
+//    normalisation: A'_t = A_t - k t and B'_t = B_t - k (n-1-t).  Since
+//    phi <= 0 and a K-term log-sum-exp exceeds its largest term by at most k,
+//    A' and B' stay <= 0 (up to rounding) with no team-wide reduction.
+//  * Forward log-sum-exp of a group: the reference is the largest term with
+//    the low word of its float64 cleared (for values <= 0 the high words order
+//    like the values, so an unsigned min finds it), plus 1.  Every exponent
+//    argument is then <= -1, computed in float64, and is rounded to a float
+//    with four integer instructions instead of a float64->float32 conversion,
+//    which shares the special-function pipe with ex2/lg2.
+//  * Backward: the exponent is the posterior itself,
+//        log2 gamma_t(s) = phi_t(s) + A'_t(h_j) + B'_t(g_b) + k(n-1) - log2 Z,
+//    taken with an offset of -1 so that the same conversion applies; one
+//    exponential per state yields both the marginal and the backward
+//    recursion  B'_{t-1}(h) = log2 sum_b 2^(log2 gamma_t - 1) - r_h - k.
+//  * Forward values needed by the backward sweep are kept per step (C = 1)
+//    as floats relative to a per-thread reference (the high word of the
+//    thread's largest group value), fetched one step ahead with cp.async;
+//    with C > 1 only every C-th step is kept (float64) and each C-segment is
+//    recomputed.
 //
-// Schedule.  One call = one launch.  A team (thread-block cluster) keeps NSEQ
-// sequences in flight and alternates their steps; each step ends with a
-// split cluster barrier whose arrive/wait brackets the other sequence's step,
-// so the barrier latency hides behind useful work.  Global stores of a step
-// (checkpoints, per-step tables, partial sums) are issued after the arrive,
-// so its release never waits for them.  The forward values needed by the
-// backward sweep are kept per step (C = 1) in a thread-private layout and
-// fetched one step ahead with cp.async; with C > 1 only every C-th step is
-// kept (float64) and each C-segment is recomputed bit-identically.
+// Schedule.  A team (thread-block cluster, one CTA, or a slice of a warp)
+// keeps NSEQ sequences in flight.  With NSEQ = 2 the steps of the two
+// sequences alternate and each step ends with a split cluster barrier whose
+// wait is deferred past the other sequence's step, so the barrier latency
+// hides behind useful work.  Global stores of a step are issued after the
+// arrive, so its release never waits for them.
 #pragma once
 #include <cfloat>
 #include <cmath>
@@ -50,10 +61,44 @@ namespace bcjr {
 namespace fbk {
 
 constexpr unsigned kFull = 0xffffffffu;
+constexpr double kMaxScaled = 1099511627776.0;       // 2^40: bound on |w'| and |c'| (every exponent stays < 2^128)
+constexpr float kNegLarge = -1.2379400392853803e27f;  // -2^90: stands for log2 0 in a group value
+
+// x <= -0.5 with |x| < 2^128: x rounded to a float (to nearest, ties away
+// from zero) with integer instructions only.  Shifted left by four, the high
+// word holds the low eight bits of the double's exponent field followed by 24
+// mantissa bits; adding one and shifting back rounds the mantissa to 23 bits
+// (a carry moves into the exponent, as it should), and the xor on the top
+// exponent bit re-biases 1023 -> 127 (896 = 0b11'1000'0000) for every
+// exponent in range.  (Truncating instead would bias every exponential
+// upwards by half a unit in the last place, which the recursions accumulate.)
+__device__ __forceinline__ float neg_d2f(double x) {
+  const uint32_t lo = static_cast<uint32_t>(__double2loint(x));
+  const uint32_t hi = static_cast<uint32_t>(__double2hiint(x));
+  const uint32_t f = (__funnelshift_l(lo, hi, 4) + 1u) >> 1;
+  return __uint_as_float((f | 0x80000000u) ^ 0x40000000u);
+}
+// v a normal negative float: the same value as a double (the inverse shuffle;
+// 0xA8000000 = sign + exponent re-bias - the float sign bit shifted down).
+__device__ __forceinline__ double neg_f2d(float v) {
+  const uint32_t f = __float_as_uint(v);
+  return __hiloint2double(static_cast<int>((f >> 3) + 0xA8000000u), static_cast<int>(f << 29));
+}
+// High word of a double as an ordering key: among values <= 0 a smaller key is
+// a larger value, and a (tiny, rounding-born) positive value has a smaller key
+// than every negative one.
+__device__ __forceinline__ uint32_t hi_key(double x) { return static_cast<uint32_t>(__double2hiint(x)); }
+__device__ __forceinline__ double from_key(uint32_t h) { return __hiloint2double(static_cast<int>(h), 0); }
+
+__device__ __forceinline__ uint32_t group_min_u32(uint32_t v, int width) {
+  if (width == 32) return __reduce_min_sync(kFull, v);
+  for (int o = width >> 1; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(kFull, v, o));
+  return v;
+}
 
 // Barrier schedule of one team.  With NSEQ = 2 on a cluster: after block b,
 // wait for the phase of block b-1 (the previous step of the other sequence)
-// and arrive for block b.  Global stores go between the two calls.
+// and arrive for block b.  Global stores go after the arrive.
 template <int CL, int NSEQ>
 struct Pipe {
   bool pending = false;
@@ -79,22 +124,6 @@ struct Pipe {
   }
 };
 
-template <int K, int CL>
-__device__ __forceinline__ float publish_max(const Team<K, CL>& tm, float* maxp_buf, float v) {
-  const float wm = group_max(v, tm.width);
-  if (tm.TS > 32 && tm.lane == 0) {
-#pragma unroll
-    for (int r = 0; r < CL; ++r) team_store<CL>(maxp_buf, r, tm.warp_in_team, wm);
-  }
-  return wm;
-}
-template <int K, int CL>
-__device__ __forceinline__ float collect_max(const Team<K, CL>& tm, const float* maxp_buf, float wm) {
-  if (tm.TS <= 32) return wm;
-  float m = -INFINITY;
-  for (int i = tm.lane; i < tm.wpt; i += 32) m = fmaxf(m, maxp_buf[i]);
-  return group_max(m, 32);
-}
 // Team-wide sum in a fixed order (every thread gets the same bits).
 template <int K, int CL>
 __device__ __forceinline__ double team_sum(const Team<K, CL>& tm, float* red, float v) {
@@ -109,6 +138,21 @@ __device__ __forceinline__ double team_sum(const Team<K, CL>& tm, float* red, fl
   for (int i = 0; i < tm.wpt; ++i) s += static_cast<double>(red[i]);
   team_sync<CL>();
   return s;
+}
+// Team-wide minimum of an unsigned key.
+template <int K, int CL>
+__device__ __forceinline__ uint32_t team_min_key(const Team<K, CL>& tm, uint32_t* red, uint32_t v) {
+  v = group_min_u32(v, tm.width);
+  if (tm.TS <= 32) return v;
+  if (tm.lane == 0) {
+#pragma unroll
+    for (int r = 0; r < CL; ++r) team_store_u32<CL>(red, r, tm.warp_in_team, v);
+  }
+  team_sync<CL>();
+  uint32_t m = 0xffffffffu;
+  for (int i = 0; i < tm.wpt; ++i) m = min(m, red[i]);
+  team_sync<CL>();
+  return m;
 }
 
 }  // namespace fbk
@@ -130,19 +174,30 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
   const int GL = tm.GL;
   // The K (k <= 2: all U*K) outputs of a forward step land in consecutive slots of one CTA.
   const bool contig = (K <= 4) && (L >= 3 * k);
+  const double kd = static_cast<double>(k);
 
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const FBSmem lay = fb_smem_layout(GL, NT, NV, NSEQ, ADJ, alias, tpc);
   unsigned char* team_base = smem_raw + static_cast<size_t>(team_in_cta) * lay.per_team;
   float* red = reinterpret_cast<float*>(smem_raw + lay.red);
+  uint32_t* redk = reinterpret_cast<uint32_t*>(smem_raw + lay.red) + 256;
 
-  float cb[U][JT][BT];
+  // Codewords of the thread's 16 states: float (for float32 sums) and scaled float64.
+  const double sqsc = p.sqsc;
+  float cf[U][JT][BT];
+  double cp[U][JT][BT];
+  bool bad_cb = false;
 #pragma unroll
   for (int u = 0; u < U; ++u)
 #pragma unroll
     for (int jj = 0; jj < JT; ++jj)
 #pragma unroll
-      for (int bb = 0; bb < BT; ++bb) cb[u][jj][bb] = __ldg(p.codebook + tm.state(u, jj, bb));
+      for (int bb = 0; bb < BT; ++bb) {
+        cf[u][jj][bb] = __ldg(p.codebook + tm.state(u, jj, bb));
+        cp[u][jj][bb] = static_cast<double>(cf[u][jj][bb]) * sqsc;
+        bad_cb |= !(fabs(cp[u][jj][bb]) <= fbk::kMaxScaled);
+      }
+  if (bad_cb) atomicOr(p.status, kDevNonFinite);
   float gc[U][JT][BT];
   if constexpr (ADJ) {
 #pragma unroll
@@ -157,7 +212,6 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
   // another's shared memory.
   if constexpr (CL > 1) cluster_sync_all();
 
-  const double sc64 = p.sc64;
   const int tvo = tm.tt * NV;  // this thread's offset in a thread-private row
   const int nsl = p.num_slots;
   const int iters = (p.N + nsl * NSEQ - 1) / (nsl * NSEQ);
@@ -166,11 +220,9 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
   struct Seq {
     int seq;
     bool act;
-    float M;      // team max of the incoming vector, subtracted on read
-    float Mpend;  // this step's max when the team fits in a warp
-    double acc;   // forward: C_t;  backward: D_t - log2 Z
-    double logZ;
-    float Dc;     // backward call: E[sum_t g_t (c(s_t) - w_hat_t)]
+    bool bad;   // an input weight was not finite or out of range
+    double K0;  // k (n-1) - log2 Z
+    float Dc;   // backward call: E[sum_t g_t (c(s_t) - w_hat_t)]
   };
 
   for (int it = 0; it < iters; ++it) {
@@ -180,34 +232,41 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
       const int s = slot + (it * NSEQ + x) * nsl;
       sq[x].act = s < p.N;
       sq[x].seq = sq[x].act ? s : p.N - 1;
-      sq[x].M = 0.f;
-      sq[x].Mpend = 0.f;
-      sq[x].acc = 0.0;
-      sq[x].logZ = 0.0;
+      sq[x].bad = false;
+      sq[x].K0 = 0.0;
       sq[x].Dc = 0.f;
     }
     fbk::Pipe<CL, NSEQ> pipe;
 
-    // ---------------- forward block: A_t -> raw A_{t+1} ----------------
-    auto alpha_block = [&](auto xc, int t) {
+    // Forward step of sequence X at step t: reads A'_t (and F~_t) from the
+    // exchange buffers, or from a0/f0 when given; when `write` is set, writes
+    // A'_{t+1} (and F~_{t+1}) to the readers' exchange buffers.  Leaves the
+    // inputs in a / f.
+    auto forward_step = [&](auto xc, int t, const double* a0, const float* f0, bool write, double* a, float* f) {
       constexpr int X = decltype(xc)::value;
       Seq& c = sq[X];
       unsigned char* sb = team_base + static_cast<size_t>(X) * lay.per_seq;
-      double* exA_r = reinterpret_cast<double*>(sb + lay.exA) + (t & 1) * GL;
+      const double* exA_r = reinterpret_cast<const double*>(sb + lay.exA) + (t & 1) * GL;
       double* exA_w = reinterpret_cast<double*>(sb + lay.exA) + ((t + 1) & 1) * GL;
-      float* exF_r = reinterpret_cast<float*>(sb + lay.exF) + (t & 1) * GL;
+      const float* exF_r = reinterpret_cast<const float*>(sb + lay.exF) + (t & 1) * GL;
       float* exF_w = reinterpret_cast<float*>(sb + lay.exF) + ((t + 1) & 1) * GL;
-      float* mp_r = reinterpret_cast<float*>(sb + lay.maxp) + (t & 1) * 128;
-      float* mp_w = reinterpret_cast<float*>(sb + lay.maxp) + ((t + 1) & 1) * 128;
-      const size_t lane_id = static_cast<size_t>(slot) * NSEQ + X;
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int jj = 0; jj < JT; ++jj) {
+          if (a0) {
+            a[u * JT + jj] = a0[u * JT + jj];
+            if constexpr (ADJ) f[u * JT + jj] = f0[u * JT + jj];
+          } else {
+            a[u * JT + jj] = (t == 0) ? 0.0 : exA_r[tm.a_read_off(u, jj)];
+            if constexpr (ADJ) f[u * JT + jj] = (t == 0) ? 0.f : exF_r[tm.a_read_off(u, jj)];
+          }
+        }
+      if (!write) return;
       const float* wrow = p.w + static_cast<size_t>(c.seq) * n;
-      if (t > 0) {
-        const float Mn = fbk::collect_max(tm, mp_r, c.Mpend);
-        c.acc += static_cast<double>(c.M);
-        c.M = Mn;
-      }
-      const double Mt = static_cast<double>(c.M);
       const float wt = __ldg(wrow + t);
+      const double wp = static_cast<double>(wt) * sqsc;
+      c.bad |= !(fabs(wp) <= fbk::kMaxScaled);
       float gt = 0.f, gw = 0.f;
       if constexpr (ADJ) {
         gt = __ldg(p.g + static_cast<size_t>(c.seq) * n + t);
@@ -220,17 +279,6 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
           asm volatile("prefetch.global.L1 [%0];" ::"l"(p.what_in + static_cast<size_t>(c.seq) * n + t + 1));
         }
       }
-      const double wt64 = static_cast<double>(wt);
-      double a[U][JT];
-      float f[U][JT];
-#pragma unroll
-      for (int u = 0; u < U; ++u)
-#pragma unroll
-        for (int jj = 0; jj < JT; ++jj) {
-          a[u][jj] = (t == 0) ? 0.0 : exA_r[tm.a_read_off(u, jj)] - Mt;
-          if constexpr (ADJ) f[u][jj] = (t == 0) ? 0.f : exF_r[tm.a_read_off(u, jj)];
-        }
-      float lmax = -INFINITY;
       double outs[U][BT];
       float fos[U][BT];
 #pragma unroll
@@ -238,25 +286,24 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
 #pragma unroll
         for (int bb = 0; bb < BT; ++bb) {
           double xv[JT];
-          float m32 = -INFINITY;
+          uint32_t key = 0xffffffffu;
 #pragma unroll
           for (int jj = 0; jj < JT; ++jj) {
-            const double d = wt64 - static_cast<double>(cb[u][jj][bb]);
-            xv[jj] = fma(-sc64 * d, d, a[u][jj]);
-            m32 = fmaxf(m32, static_cast<float>(xv[jj]));
+            const double d = wp - cp[u][jj][bb];
+            xv[jj] = fma(-d, d, a[u * JT + jj]);
+            key = min(key, fbk::hi_key(xv[jj]));
           }
           if constexpr (K >= 8) {
 #pragma unroll
-            for (int o = TL::NBT; o < TL::TPU; o <<= 1) m32 = fmaxf(m32, __shfl_xor_sync(fbk::kFull, m32, o));
+            for (int o = TL::NBT; o < TL::TPU; o <<= 1) key = min(key, __shfl_xor_sync(fbk::kFull, key, o));
           }
-          // reference point: the largest term rounded to float (any nearby value is exact for the LSE)
-          const double m = static_cast<double>(m32);
+          const double ref = fbk::from_key(key) + 1.0;
           float s = 0.f, num = 0.f;
 #pragma unroll
           for (int jj = 0; jj < JT; ++jj) {
-            const float e = ex2f(static_cast<float>(xv[jj] - m));
+            const float e = ex2f(fbk::neg_d2f(xv[jj] - ref));
             s += e;
-            if constexpr (ADJ) num = fmaf(e, f[u][jj] + fmaf(gt, cb[u][jj][bb], -gw), num);
+            if constexpr (ADJ) num = fmaf(e, f[u * JT + jj] + fmaf(gt, cf[u][jj][bb], -gw), num);
           }
           if constexpr (K >= 8) {
 #pragma unroll
@@ -265,73 +312,89 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
               if constexpr (ADJ) num += __shfl_xor_sync(fbk::kFull, num, o);
             }
           }
-          outs[u][bb] = m + static_cast<double>(lg2f(s));
+          outs[u][bb] = static_cast<double>(lg2f(s)) + (ref - kd);
           if constexpr (ADJ) fos[u][bb] = num * rcpf(s);
-          lmax = fmaxf(lmax, static_cast<float>(outs[u][bb]));
         }
       }
-      if (tm.a_writer) {
-        if (contig) {
-          // k <= 2: the U*K outputs are consecutive slots of one CTA.
-          uint32_t r;
-          int off;
-          tm.a_dest(tm.a_out_index(0, 0), r, off);
+      if (!tm.a_writer) return;
+      if (contig) {
+        uint32_t r;
+        int off;
+        tm.a_dest(tm.a_out_index(0, 0), r, off);
 #pragma unroll
-          for (int v = 0; v < U * BT; v += 2) {
-            const double o0 = outs[v / BT][v % BT], o1 = outs[(v + 1) / BT][(v + 1) % BT];
-            if constexpr (CL == 1) {
-              *reinterpret_cast<double2*>(exA_w + off + v) = make_double2(o0, o1);
-            } else {
-              st_cluster_v2f64(exA_w + off + v, r, o0, o1);
-            }
+        for (int v = 0; v < U * BT; v += 2) {
+          const double o0 = outs[v / BT][v % BT], o1 = outs[(v + 1) / BT][(v + 1) % BT];
+          if constexpr (CL == 1) {
+            *reinterpret_cast<double2*>(exA_w + off + v) = make_double2(o0, o1);
+            if constexpr (ADJ)
+              *reinterpret_cast<float2*>(exF_w + off + v) =
+                  make_float2(fos[v / BT][v % BT], fos[(v + 1) / BT][(v + 1) % BT]);
+          } else {
+            st_cluster_v2f64(exA_w + off + v, r, o0, o1);
             if constexpr (ADJ) {
               team_store<CL>(exF_w, r, off + v, fos[v / BT][v % BT]);
               team_store<CL>(exF_w, r, off + v + 1, fos[(v + 1) / BT][(v + 1) % BT]);
             }
           }
-        } else {
-#pragma unroll
-          for (int u = 0; u < U; ++u)
-#pragma unroll
-            for (int bb = 0; bb < BT; ++bb) {
-              uint32_t r;
-              int off;
-              tm.a_dest(tm.a_out_index(u, bb), r, off);
-              team_store_f64<CL>(exA_w, r, off, outs[u][bb]);
-              if constexpr (ADJ) team_store<CL>(exF_w, r, off, fos[u][bb]);
-            }
         }
       } else {
-        lmax = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+          for (int bb = 0; bb < BT; ++bb) {
+            uint32_t r;
+            int off;
+            tm.a_dest(tm.a_out_index(u, bb), r, off);
+            team_store_f64<CL>(exA_w, r, off, outs[u][bb]);
+            if constexpr (ADJ) team_store<CL>(exF_w, r, off, fos[u][bb]);
+          }
       }
-      c.Mpend = fbk::publish_max(tm, mp_w, lmax);
+    };
+
+    // Checkpoint row of A'_t (floats relative to the thread's reference) and F~_t.
+    auto store_checkpoint = [&](const double* a, const float* f, float* ckrow, uint32_t* ckkey, float* ckrowF) {
+      uint32_t key = 0xffffffffu;
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int jj = 0; jj < JT; ++jj) key = min(key, fbk::hi_key(a[u * JT + jj]));
+      const double R1 = fbk::from_key(key) + 1.0;
+#pragma unroll
+      for (int v = 0; v < NV; v += 4) {
+        *reinterpret_cast<float4*>(ckrow + v) = make_float4(
+            fbk::neg_d2f(a[v] - R1), fbk::neg_d2f(a[(v + 1)] - R1),
+            fbk::neg_d2f(a[(v + 2)] - R1), fbk::neg_d2f(a[(v + 3)] - R1));
+        if constexpr (ADJ)
+          *reinterpret_cast<float4*>(ckrowF + v) =
+              make_float4(f[v], f[(v + 1)], f[(v + 2)],
+                          f[(v + 3)]);
+      }
+      *ckkey = key;
+    };
+
+    // ---------------- forward sweep ----------------
+    auto alpha_block = [&](auto xc, int t) {
+      constexpr int X = decltype(xc)::value;
+      const size_t lane_id = static_cast<size_t>(slot) * NSEQ + X;
+      double a[NV];
+      float f[NV];
+      forward_step(xc, t, nullptr, nullptr, true, a, f);
       pipe.before_stores();
       // ---- this step's global stores (outside the barrier's release) ----
       if (C == 1) {
-        float* row = p.ck + lane_id * p.ck_stride + static_cast<size_t>(t) * p.row + tvo;
-        float* rowF = ADJ ? p.ckF + lane_id * p.ck_stride + static_cast<size_t>(t) * p.row + tvo : nullptr;
-#pragma unroll
-        for (int v = 0; v < NV; v += 4) {
-          *reinterpret_cast<float4*>(row + v) = make_float4(
-              static_cast<float>(a[v / JT][v % JT]), static_cast<float>(a[(v + 1) / JT][(v + 1) % JT]),
-              static_cast<float>(a[(v + 2) / JT][(v + 2) % JT]), static_cast<float>(a[(v + 3) / JT][(v + 3) % JT]));
-          if constexpr (ADJ)
-            *reinterpret_cast<float4*>(rowF + v) =
-                make_float4(f[v / JT][v % JT], f[(v + 1) / JT][(v + 1) % JT], f[(v + 2) / JT][(v + 2) % JT],
-                            f[(v + 3) / JT][(v + 3) % JT]);
-        }
-      } else if (t % C == 0) {
+        store_checkpoint(a, f, p.ck + lane_id * p.ck_stride + static_cast<size_t>(t) * p.row + tvo,
+                         p.ckR + lane_id * p.ckR_stride + static_cast<size_t>(t) * TS + tm.tt,
+                         ADJ ? p.ckF + lane_id * p.ck_stride + static_cast<size_t>(t) * p.row + tvo : nullptr);
+      } else if (t % C == 0) {  // exact float64 forward values at the segment starts
         double* row = p.ck64 + lane_id * p.ck64_stride + static_cast<size_t>(t / C) * p.row + tvo;
         float* rowF = ADJ ? p.ckF64 + lane_id * p.ck64_stride + static_cast<size_t>(t / C) * p.row + tvo : nullptr;
 #pragma unroll
-        for (int v = 0; v < NV; ++v) {
-          row[v] = a[v / JT][v % JT];
-          if constexpr (ADJ) rowF[v] = f[v / JT][v % JT];
-        }
-      }
-      if (tm.tt == 0) {
-        p.Mtab[lane_id * p.tab_stride + t] = c.M;
-        p.Ctab[lane_id * p.tab_stride + t] = c.acc + Mt;
+        for (int u = 0; u < U; ++u)
+#pragma unroll
+          for (int jj = 0; jj < JT; ++jj) {
+            row[u * JT + jj] = a[u * JT + jj];
+            if constexpr (ADJ) rowF[u * JT + jj] = f[u * JT + jj];
+          }
       }
       pipe.after_stores();
     };
@@ -342,154 +405,97 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
     }
     pipe.drain();
 
-    // log2 Z = C_n + log2 sum_g 2^{A_n(g)};  D = E[sum_t g_t (c(s_t) - w_hat_t)] (backward call).
+    // log2 Z = k n + log2 sum_g 2^{A'_n(g)};  D = E[sum_t g_t (c(s_t) - w_hat_t)] (backward call).
     auto finish_forward = [&](auto xc) {
       constexpr int X = decltype(xc)::value;
       Seq& c = sq[X];
       unsigned char* sb = team_base + static_cast<size_t>(X) * lay.per_seq;
       const double* exA_r = reinterpret_cast<const double*>(sb + lay.exA) + (n & 1) * GL;
       const float* exF_r = reinterpret_cast<const float*>(sb + lay.exF) + (n & 1) * GL;
-      const float Mn = fbk::collect_max(tm, reinterpret_cast<float*>(sb + lay.maxp) + (n & 1) * 128, c.Mpend);
-      const double Cn = c.acc + static_cast<double>(c.M);
+      double av[U][JT];
+      uint32_t key = 0xffffffffu;
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int jj = 0; jj < JT; ++jj) {
+          av[u][jj] = exA_r[tm.a_read_off(u, jj)];
+          if (tm.b_writer) key = min(key, fbk::hi_key(av[u][jj]));  // one reader per group value
+        }
+      const double Rt = fbk::from_key(fbk::team_min_key(tm, redk, key));
       float s1 = 0.f, s2 = 0.f;
-      if (tm.b_writer) {  // one reader per group value
+      if (tm.b_writer) {
 #pragma unroll
         for (int u = 0; u < U; ++u)
 #pragma unroll
           for (int jj = 0; jj < JT; ++jj) {
-            const float e = ex2f(static_cast<float>(exA_r[tm.a_read_off(u, jj)] - static_cast<double>(Mn)));
+            const float e = ex2f(static_cast<float>(av[u][jj] - Rt));
             s1 += e;
             if constexpr (ADJ) s2 = fmaf(e, exF_r[tm.a_read_off(u, jj)], s2);
           }
       }
       const double S1 = fbk::team_sum(tm, red, s1);
       const double S2 = ADJ ? fbk::team_sum(tm, red + 128, s2) : 0.0;
-      c.logZ = Cn + static_cast<double>(Mn) + log2(S1);
+      const double log2Z = kd * n + Rt + log2(S1);
+      c.K0 = kd * (n - 1) - log2Z;
       c.Dc = ADJ ? static_cast<float>(S2 / S1) : 0.f;
       if (tm.tt == 0 && c.act) {
-        if (!isfinite(c.logZ)) atomicOr(p.status, kDevNonFinite);
+        const bool ok = isfinite(log2Z) && !c.bad;
+        if (!ok) atomicOr(p.status, kDevNonFinite);
         if constexpr (!ADJ) {
-          if (p.log_z) p.log_z[c.seq] = static_cast<float>(c.logZ * 0.69314718055994530942);
+          if (p.log_z) p.log_z[c.seq] = ok ? static_cast<float>(log2Z * 0.69314718055994530942) : NAN;
         }
       }
-      c.M = 0.f;
-      c.Mpend = 0.f;
-      c.acc = -c.logZ;  // backward: D_t - log2 Z with D_{n-1} = 0
     };
     finish_forward(std::integral_constant<int, 0>{});
     if constexpr (NSEQ == 2) finish_forward(std::integral_constant<int, 1>{});
     team_sync<CL>();
 
-    // ---------------- backward block: B_t -> gamma_t, raw B_{t-1} ----------------
+    // ---------------- backward sweep ----------------
+    // C > 1: recompute the forward values of the segment [t0, t1] into the ring
+    // (rows 0 .. t1-t0, same format as the C = 1 rows).
+    auto recompute_segment = [&](int t0, int t1) {
+      for (int tp = t0; tp <= t1; ++tp) {
+        auto one = [&](auto xc) {
+          constexpr int X = decltype(xc)::value;
+          const size_t lane_id = static_cast<size_t>(slot) * NSEQ + X;
+          const double* c64 = p.ck64 + lane_id * p.ck64_stride + static_cast<size_t>(t0 / C) * p.row + tvo;
+          const float* cF64 =
+              ADJ ? p.ckF64 + lane_id * p.ck64_stride + static_cast<size_t>(t0 / C) * p.row + tvo : nullptr;
+          double a[NV];
+          float f[NV];
+          forward_step(xc, tp, tp == t0 ? c64 : nullptr, tp == t0 ? cF64 : nullptr, tp < t1, a, f);
+          store_checkpoint(a, f, p.ck + lane_id * p.ck_stride + static_cast<size_t>(tp - t0) * p.row + tvo,
+                           p.ckR + lane_id * p.ckR_stride + static_cast<size_t>(tp - t0) * TS + tm.tt,
+                           ADJ ? p.ckF + lane_id * p.ck_stride + static_cast<size_t>(tp - t0) * p.row + tvo : nullptr);
+        };
+        one(std::integral_constant<int, 0>{});
+        if constexpr (NSEQ == 2) one(std::integral_constant<int, 1>{});
+        team_sync<CL>();
+      }
+    };
+
     auto beta_block = [&](auto xc, int t) {
       constexpr int X = decltype(xc)::value;
       Seq& c = sq[X];
       unsigned char* sb = team_base + static_cast<size_t>(X) * lay.per_seq;
       const size_t lane_id = static_cast<size_t>(slot) * NSEQ + X;
       const float* wrow = p.w + static_cast<size_t>(c.seq) * n;
-      const double* ctab = p.Ctab + lane_id * p.tab_stride;
-      // C > 1: recompute this C-segment's forward values (one sequence in flight).
-      if (C > 1 && (t == n - 1 || (t + 1) % C == 0)) {
-        const int t0 = t - (t % C);
-        const float* mtab = p.Mtab + lane_id * p.tab_stride;
-        for (int tp = t0; tp <= t; ++tp) {
-          double* exA_r = reinterpret_cast<double*>(sb + lay.exA) + (tp & 1) * GL;
-          double* exA_w = reinterpret_cast<double*>(sb + lay.exA) + ((tp + 1) & 1) * GL;
-          float* exF_r = reinterpret_cast<float*>(sb + lay.exF) + (tp & 1) * GL;
-          float* exF_w = reinterpret_cast<float*>(sb + lay.exF) + ((tp + 1) & 1) * GL;
-          const double Mtp = static_cast<double>(mtab[tp]);
-          float* ring = p.ck + lane_id * p.ck_stride + static_cast<size_t>(tp - t0) * p.row + tvo;
-          float* ringF = ADJ ? p.ckF + lane_id * p.ck_stride + static_cast<size_t>(tp - t0) * p.row + tvo : nullptr;
-          const double* c64 = p.ck64 + lane_id * p.ck64_stride + static_cast<size_t>(t0 / C) * p.row + tvo;
-          const float* cF64 = ADJ ? p.ckF64 + lane_id * p.ck64_stride + static_cast<size_t>(t0 / C) * p.row + tvo
-                                  : nullptr;
-          double a[U][JT];
-          float f[U][JT];
-#pragma unroll
-          for (int u = 0; u < U; ++u)
-#pragma unroll
-            for (int jj = 0; jj < JT; ++jj) {
-              if (tp == t0) {
-                a[u][jj] = (tp == 0) ? 0.0 : c64[u * JT + jj];
-                if constexpr (ADJ) f[u][jj] = (tp == 0) ? 0.f : cF64[u * JT + jj];
-              } else {
-                a[u][jj] = exA_r[tm.a_read_off(u, jj)] - Mtp;
-                if constexpr (ADJ) f[u][jj] = exF_r[tm.a_read_off(u, jj)];
-              }
-              ring[u * JT + jj] = static_cast<float>(a[u][jj]);
-              if constexpr (ADJ) ringF[u * JT + jj] = f[u][jj];
-            }
-          if (tp < t) {
-            const double wt64 = static_cast<double>(__ldg(wrow + tp));
-            float gt = 0.f, gw = 0.f;
-            if constexpr (ADJ) {
-              gt = __ldg(p.g + static_cast<size_t>(c.seq) * n + tp);
-              gw = gt * __ldg(p.what_in + static_cast<size_t>(c.seq) * n + tp);
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-#pragma unroll
-              for (int bb = 0; bb < BT; ++bb) {
-                double xv[JT];
-                float m32 = -INFINITY;
-#pragma unroll
-                for (int jj = 0; jj < JT; ++jj) {
-                  const double d = wt64 - static_cast<double>(cb[u][jj][bb]);
-                  xv[jj] = fma(-sc64 * d, d, a[u][jj]);
-                  m32 = fmaxf(m32, static_cast<float>(xv[jj]));
-                }
-                if constexpr (K >= 8) {
-#pragma unroll
-                  for (int o = TL::NBT; o < TL::TPU; o <<= 1) m32 = fmaxf(m32, __shfl_xor_sync(fbk::kFull, m32, o));
-                }
-                const double m = static_cast<double>(m32);
-                float s = 0.f, num = 0.f;
-#pragma unroll
-                for (int jj = 0; jj < JT; ++jj) {
-                  const float e = ex2f(static_cast<float>(xv[jj] - m));
-                  s += e;
-                  if constexpr (ADJ) num = fmaf(e, f[u][jj] + fmaf(gt, cb[u][jj][bb], -gw), num);
-                }
-                if constexpr (K >= 8) {
-#pragma unroll
-                  for (int o = TL::NBT; o < TL::TPU; o <<= 1) {
-                    s += __shfl_xor_sync(fbk::kFull, s, o);
-                    if constexpr (ADJ) num += __shfl_xor_sync(fbk::kFull, num, o);
-                  }
-                }
-                if (tm.a_writer) {
-                  uint32_t r;
-                  int off;
-                  tm.a_dest(tm.a_out_index(u, bb), r, off);
-                  team_store_f64<CL>(exA_w, r, off, m + static_cast<double>(lg2f(s)));
-                  if constexpr (ADJ) team_store<CL>(exF_w, r, off, num * rcpf(s));
-                }
-              }
-            }
-          }
-          team_sync<CL>();
-        }
-      }
-
       const double* exB_r = reinterpret_cast<const double*>(sb + lay.exB) + (t & 1) * GL;
       double* exB_w = reinterpret_cast<double*>(sb + lay.exB) + ((t + 1) & 1) * GL;  // (t-1) & 1
       const float* exBt_r = reinterpret_cast<const float*>(sb + lay.exBt) + (t & 1) * GL;
       float* exBt_w = reinterpret_cast<float*>(sb + lay.exBt) + ((t + 1) & 1) * GL;
-      float* mp_r = reinterpret_cast<float*>(sb + lay.maxp) + (t & 1) * 128;
-      float* mp_w = reinterpret_cast<float*>(sb + lay.maxp) + ((t + 1) & 1) * 128;
-      float* stg_r = reinterpret_cast<float*>(smem_raw + lay.stage) + (static_cast<size_t>(X * 2 + (t & 1)) * NT + threadIdx.x) * NV;
-      float* stg_w = reinterpret_cast<float*>(smem_raw + lay.stage) + (static_cast<size_t>(X * 2 + ((t + 1) & 1)) * NT + threadIdx.x) * NV;
-      float* stgF_r = reinterpret_cast<float*>(smem_raw + lay.stageF) + (static_cast<size_t>(X * 2 + (t & 1)) * NT + threadIdx.x) * NV;
-      float* stgF_w = reinterpret_cast<float*>(smem_raw + lay.stageF) + (static_cast<size_t>(X * 2 + ((t + 1) & 1)) * NT + threadIdx.x) * NV;
-      if (t < n - 1) {
-        const float Mn = fbk::collect_max(tm, mp_r, c.Mpend);
-        c.acc += static_cast<double>(c.M);
-        c.M = Mn;
-      }
-      const double Mbt = static_cast<double>(c.M);
-      // forward values A_t(h) - M_t (and F_t(h)) at the thread's groups h
+      // forward values of step t as stored, and the thread's reference key
       float ra[NV], fa[NV];
+      uint32_t rkey;
       if (C == 1) {
+        const size_t par_r = static_cast<size_t>(X * 2 + (t & 1)) * NT + threadIdx.x;
+        const size_t par_w = static_cast<size_t>(X * 2 + ((t + 1) & 1)) * NT + threadIdx.x;
+        float* stg_r = reinterpret_cast<float*>(smem_raw + lay.stage) + par_r * NV;
+        float* stg_w = reinterpret_cast<float*>(smem_raw + lay.stage) + par_w * NV;
+        float* stgF_r = reinterpret_cast<float*>(smem_raw + lay.stageF) + par_r * NV;
+        float* stgF_w = reinterpret_cast<float*>(smem_raw + lay.stageF) + par_w * NV;
+        uint32_t* stgK_r = reinterpret_cast<uint32_t*>(smem_raw + lay.stageK) + par_r;
+        uint32_t* stgK_w = reinterpret_cast<uint32_t*>(smem_raw + lay.stageK) + par_w;
         if constexpr (NSEQ == 2) {
           cp_async_wait<1>();
         } else {
@@ -510,29 +516,38 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
             fa[v + 3] = f4.w;
           }
         }
+        rkey = *stgK_r;
         if (t >= 1) {
           const float* src = p.ck + lane_id * p.ck_stride + static_cast<size_t>(t - 1) * p.row + tvo;
-          const float* srcF = ADJ ? p.ckF + lane_id * p.ck_stride + static_cast<size_t>(t - 1) * p.row + tvo : nullptr;
+          const float* srcF =
+              ADJ ? p.ckF + lane_id * p.ck_stride + static_cast<size_t>(t - 1) * p.row + tvo : nullptr;
 #pragma unroll
           for (int v = 0; v < NV; v += 4) {
             cp_async16(stg_w + v, src + v);
             if constexpr (ADJ) cp_async16(stgF_w + v, srcF + v);
           }
+          cp_async4(stgK_w, p.ckR + lane_id * p.ckR_stride + static_cast<size_t>(t - 1) * TS + tm.tt);
         }
         cp_async_commit();
       } else {
         const int t0 = t - (t % C);
         const float* ring = p.ck + lane_id * p.ck_stride + static_cast<size_t>(t - t0) * p.row + tvo;
-        const float* ringF = ADJ ? p.ckF + lane_id * p.ck_stride + static_cast<size_t>(t - t0) * p.row + tvo : nullptr;
+        const float* ringF =
+            ADJ ? p.ckF + lane_id * p.ck_stride + static_cast<size_t>(t - t0) * p.row + tvo : nullptr;
 #pragma unroll
         for (int v = 0; v < NV; ++v) {
           ra[v] = ring[v];
           if constexpr (ADJ) fa[v] = ringF[v];
         }
+        rkey = p.ckR[lane_id * p.ckR_stride + static_cast<size_t>(t - t0) * TS + tm.tt];
       }
-      const double kap = ctab[t] + Mbt + c.acc;  // C_{t+1} + M'_t + D_t - log2 Z
+      // r_j = A'_t(h_j) + k(n-1) - log2 Z - 1, so that log2 gamma_t(s) - 1 = phi_t(s) + B'_t(g_b) + r_j
+      const double RK = fbk::from_key(rkey) + c.K0;
+      double rp[NV];
+#pragma unroll
+      for (int v = 0; v < NV; ++v) rp[v] = fbk::neg_f2d(ra[v]) + RK;
       const float wt = __ldg(wrow + t);
-      const double wt64 = static_cast<double>(wt);
+      const double wp = static_cast<double>(wt) * sqsc;
       float gt = 0.f, gw = 0.f;
       if constexpr (ADJ) {
         gt = __ldg(p.g + static_cast<size_t>(c.seq) * n + t);
@@ -540,25 +555,27 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
       }
       if (t >= 1 && tm.lane == 0) {
         asm volatile("prefetch.global.L1 [%0];" ::"l"(wrow + t - 1));
-        asm volatile("prefetch.global.L1 [%0];" ::"l"(ctab + t - 1));
         if constexpr (ADJ) {
           asm volatile("prefetch.global.L1 [%0];" ::"l"(p.g + static_cast<size_t>(c.seq) * n + t - 1));
           asm volatile("prefetch.global.L1 [%0];" ::"l"(p.what_in + static_cast<size_t>(c.seq) * n + t - 1));
         }
       }
-      // incoming B_t (normalised) at the thread's successor groups (q << k) | b
+      // incoming B'_t at the thread's successor groups (q << k) | b
       double bv[U][BT];
       float btl[U][BT];
 #pragma unroll
       for (int u = 0; u < U; ++u)
 #pragma unroll
         for (int bb = 0; bb < BT; ++bb) {
-          bv[u][bb] = (t == n - 1) ? 0.0 : exB_r[tm.b_read_off(u, bb)] - Mbt;
+          bv[u][bb] = (t == n - 1) ? 0.0 : exB_r[tm.b_read_off(u, bb)];
           if constexpr (ADJ) btl[u][bb] = (t == n - 1) ? 0.f : exBt_r[tm.b_read_off(u, bb)];
         }
-      const float tw = p.two_over_T * wt;
+      // Inactive (padding) sequences contribute nothing to the codebook gradient.
+      const float actf = c.act ? 1.f : 0.f;
+      const float gta = gt * actf;
+      const float m2T = -p.two_over_T * actf;
+      const float twa = p.two_over_T * wt * actf;
       float acc0 = 0.f, acc1 = 0.f;
-      float lmax = -INFINITY;
       float* mrow = (!ADJ && p.marginals && c.act)
                         ? p.marginals + (static_cast<size_t>(c.seq) * n + t) * static_cast<size_t>(S)
                         : nullptr;
@@ -566,27 +583,28 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
       for (int u = 0; u < U; ++u) {
 #pragma unroll
         for (int jj = 0; jj < JT; ++jj) {
-          const double r = static_cast<double>(ra[u * JT + jj]) + kap;
+          const double r = rp[u * JT + jj];
           float s = 0.f, bnum = 0.f;
           const float fbase = ADJ ? fa[u * JT + jj] - c.Dc : 0.f;
 #pragma unroll
           for (int bb = 0; bb < BT; ++bb) {
-            const float cv = cb[u][jj][bb];
-            const double d = wt64 - static_cast<double>(cv);
-            const float gam = ex2f(static_cast<float>(fma(-sc64 * d, d, bv[u][bb]) + r));  // gamma_t(s)
-            s += gam;
+            const float cv = cf[u][jj][bb];
+            const double d = wp - cp[u][jj][bb];
+            const float e = ex2f(fbk::neg_d2f(fma(-d, d, bv[u][bb] + r)));  // gamma_t(s) / 2
+            s += e;
             if constexpr (!ADJ) {
-              acc0 = fmaf(gam, cv, acc0);
-              acc1 += gam;
-              if (mrow) mrow[tm.state(u, jj, bb)] = gam;
+              acc0 = fmaf(e, cv, acc0);
+              if (mrow) mrow[tm.state(u, jj, bb)] = e + e;
             } else {
               const float eps = fmaf(gt, cv, -gw) + btl[u][bb];
-              bnum = fmaf(gam, eps, bnum);
-              const float psi = gam * (fbase + eps);
+              const float ge = e * eps;
+              bnum += ge;
+              const float psi = fmaf(e, fbase, ge);  // psi_t(s) / 2
               acc0 = fmaf(psi, cv, acc0);
-              gc[u][jj][bb] += c.act ? fmaf(gt, gam, psi * fmaf(-p.two_over_T, cv, tw)) : 0.f;
+              gc[u][jj][bb] += fmaf(gta, e, psi * fmaf(m2T, cv, twa));
             }
           }
+          if constexpr (!ADJ) acc1 += s;  // this thread's states only
           if constexpr (K >= 8) {
 #pragma unroll
             for (int o = 1; o < TL::NBT; o <<= 1) {
@@ -595,19 +613,17 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
             }
           }
           if (t >= 1 && tm.b_writer) {
-            const double out = (s > 0.f) ? static_cast<double>(lg2f(s)) - r : -INFINITY;
+            const double out = static_cast<double>(s > 0.f ? lg2f(s) : fbk::kNegLarge) - (r + kd);
             uint32_t rk;
             int off;
             tm.b_dest(tm.b_out_index(u, jj), rk, off);
             team_store_f64<CL>(exB_w, rk, off, out);
             if constexpr (ADJ) team_store<CL>(exBt_w, rk, off, (s > 0.f) ? bnum * rcpf(s) : 0.f);
-            lmax = fmaxf(lmax, static_cast<float>(out));
           }
         }
       }
       const float v0 = group_sum(acc0, tm.width);
       const float v1 = ADJ ? 0.f : group_sum(acc1, tm.width);
-      if (t >= 1) c.Mpend = fbk::publish_max(tm, mp_w, lmax);
       pipe.before_stores();
       if ((tm.lane & (tm.width - 1)) == 0) {
         float* pr = p.part + lane_id * p.part_stride + static_cast<size_t>(t) * 2 * tm.wpt;
@@ -622,10 +638,10 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
 #pragma unroll
       for (int x = 0; x < NSEQ; ++x) {
         const size_t lane_id = static_cast<size_t>(slot) * NSEQ + x;
-        float* stg = reinterpret_cast<float*>(smem_raw + lay.stage) +
-                     (static_cast<size_t>(x * 2 + ((n - 1) & 1)) * NT + threadIdx.x) * NV;
-        float* stgF = reinterpret_cast<float*>(smem_raw + lay.stageF) +
-                      (static_cast<size_t>(x * 2 + ((n - 1) & 1)) * NT + threadIdx.x) * NV;
+        const size_t par = static_cast<size_t>(x * 2 + ((n - 1) & 1)) * NT + threadIdx.x;
+        float* stg = reinterpret_cast<float*>(smem_raw + lay.stage) + par * NV;
+        float* stgF = reinterpret_cast<float*>(smem_raw + lay.stageF) + par * NV;
+        uint32_t* stgK = reinterpret_cast<uint32_t*>(smem_raw + lay.stageK) + par;
         const float* src = p.ck + lane_id * p.ck_stride + static_cast<size_t>(n - 1) * p.row + tvo;
         const float* srcF = ADJ ? p.ckF + lane_id * p.ck_stride + static_cast<size_t>(n - 1) * p.row + tvo : nullptr;
 #pragma unroll
@@ -633,10 +649,15 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
           cp_async16(stg + v, src + v);
           if constexpr (ADJ) cp_async16(stgF + v, srcF + v);
         }
+        cp_async4(stgK, p.ckR + lane_id * p.ckR_stride + static_cast<size_t>(n - 1) * TS + tm.tt);
         cp_async_commit();
       }
     }
     for (int t = n - 1; t >= 0; --t) {
+      if (C > 1 && (t == n - 1 || (t + 1) % C == 0)) {
+        pipe.drain();
+        recompute_segment(t - (t % C), t);
+      }
       beta_block(std::integral_constant<int, 0>{}, t);
       if constexpr (NSEQ == 2) beta_block(std::integral_constant<int, 1>{}, t);
     }
@@ -657,7 +678,7 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
         if constexpr (!ADJ) {
           p.w_hat[static_cast<size_t>(sq[x].seq) * n + t] = v0 / v1;
         } else {
-          p.grad_w[static_cast<size_t>(sq[x].seq) * n + t] = p.two_over_T * v0;
+          p.grad_w[static_cast<size_t>(sq[x].seq) * n + t] = 2.f * p.two_over_T * v0;  // v0 sums psi/2 * c
         }
       }
     }
@@ -671,7 +692,7 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
 #pragma unroll
       for (int jj = 0; jj < JT; ++jj)
 #pragma unroll
-        for (int bb = 0; bb < BT; ++bb) gp[tm.state(u, jj, bb)] = gc[u][jj][bb];
+        for (int bb = 0; bb < BT; ++bb) gp[tm.state(u, jj, bb)] = 2.f * gc[u][jj][bb];  // gc holds halves
   }
   if constexpr (CL > 1) cluster_sync_all();  // no CTA leaves while its shared memory may be addressed
 }
