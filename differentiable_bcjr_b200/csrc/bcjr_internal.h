@@ -9,7 +9,7 @@ namespace bcjr {
 // Device-side error bits, OR-ed into the status word at the head of the workspace.
 enum : int {
   kDevNonFinite = 1,   // log Z (or a Viterbi metric) came out NaN or infinite
-  kDevTimeout = 2,     // a bounded wait gave up
+  kDevTimeout = 2,     // a bounded wait gave up (the results of the call are not valid)
 };
 
 // Geometry of one launch over the bitshift trellis (host-computed).
@@ -63,7 +63,7 @@ struct FBParams {
 // CTA: a reduction scratch and the thread-private staging of the forward
 // values read by the backward sweep (values, reference words, accumulators).
 struct FBSmem {
-  uint32_t exA, exF, exB, exBt, per_seq, per_team, red, stage, stageK, stageF, total;
+  uint32_t exA, exF, exB, exBt, mbar, per_seq, per_team, red, stage, stageK, stageF, total;
 };
 __host__ __device__ inline FBSmem fb_smem_layout(int GL, int NT, int NV, int nseq, bool adj, bool alias,
                                                  int teams_per_cta) {
@@ -78,6 +78,8 @@ __host__ __device__ inline FBSmem fb_smem_layout(int GL, int NT, int NV, int nse
   l.exBt = alias ? l.exF : o;
   if (!alias && adj) o += 2u * GL * 4u;
   o = (o + 15u) & ~15u;
+  l.mbar = o;  // 2 sets (forward / backward buffers) x 2 parities of 8-byte mbarriers
+  o += 32u;
   l.per_seq = o;
   l.per_team = static_cast<uint32_t>(nseq) * o;
   l.red = static_cast<uint32_t>(teams_per_cta) * l.per_team;

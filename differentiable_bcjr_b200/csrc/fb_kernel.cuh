@@ -99,6 +99,9 @@ __device__ __forceinline__ uint32_t group_min_u32(uint32_t v, int width) {
 // Barrier schedule of one team.  With NSEQ = 2 on a cluster: after block b,
 // wait for the phase of block b-1 (the previous step of the other sequence)
 // and arrive for block b.  Global stores go after the arrive.
+// On a cluster the exchanged data travel with st.async and are awaited on
+// mbarriers, so this barrier orders execution only (every read of a buffer
+// before its overwrite two steps later) and carries no memory fence.
 template <int CL, int NSEQ>
 struct Pipe {
   bool pending = false;
@@ -106,19 +109,19 @@ struct Pipe {
     if constexpr (CL == 1) {
       __syncthreads();
     } else if constexpr (NSEQ == 1) {
-      cluster_arrive();
+      cluster_arrive_relaxed();
     } else {
-      if (pending) cluster_wait();
-      cluster_arrive();
+      if (pending) cluster_wait_plain();
+      cluster_arrive_relaxed();
       pending = true;
     }
   }
   __device__ __forceinline__ void after_stores() {
-    if constexpr (CL > 1 && NSEQ == 1) cluster_wait();
+    if constexpr (CL > 1 && NSEQ == 1) cluster_wait_plain();
   }
   __device__ __forceinline__ void drain() {
     if constexpr (CL > 1 && NSEQ == 2) {
-      if (pending) cluster_wait();
+      if (pending) cluster_wait_plain();
       pending = false;
     }
   }
@@ -208,8 +211,42 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
         for (int bb = 0; bb < BT; ++bb) gc[u][jj][bb] = 0.f;
   }
 
-  // Every CTA of the cluster must be running before any of them writes into
-  // another's shared memory.
+  // Exchange mbarriers (cluster teams): per sequence in flight, one per
+  // buffer set (forward, backward) and parity; armed each step by thread 0
+  // with the bytes the CTA is about to receive.  With C == 1 the backward
+  // sweep reuses the forward buffers and their mbarriers.
+  const int setB = alias ? 0 : 1;
+  const uint32_t xbytes = static_cast<uint32_t>(GL) * (ADJ ? 12u : 8u);
+  auto mbar = [&](int X, int set, int par) {
+    return reinterpret_cast<uint64_t*>(team_base + static_cast<size_t>(X) * lay.per_seq + lay.mbar) + set * 2 + par;
+  };
+  uint32_t ph[NSEQ];  // parity of the next phase to wait for, bit (set * 2 + par)
+#pragma unroll
+  for (int x = 0; x < NSEQ; ++x) ph[x] = 0;
+  bool timed_out = false;  // after one wait gave up, no further waits (the call's results are void)
+  if constexpr (CL > 1) {
+    if (threadIdx.x == 0) {
+#pragma unroll
+      for (int x = 0; x < NSEQ; ++x)
+        for (int i = 0; i < 4; ++i) mbar_init(mbar(x, i >> 1, i & 1), 1);
+      mbar_init_fence();
+    }
+  }
+  auto xwait = [&](int X, int set, int par) {
+    if constexpr (CL > 1) {
+      const int bit = set * 2 + par;
+      if (!timed_out) timed_out = !mbar_wait(mbar(X, set, par), (ph[X] >> bit) & 1u, p.status, kDevTimeout);
+      ph[X] ^= 1u << bit;
+    }
+  };
+  auto xarm = [&](int X, int set, int par) {
+    if constexpr (CL > 1) {
+      if (threadIdx.x == 0) mbar_arm(mbar(X, set, par), xbytes);
+    }
+  };
+
+  // Every CTA of the cluster must be running (and its mbarriers initialised)
+  // before any of them writes into another's shared memory.
   if constexpr (CL > 1) cluster_sync_all();
 
   const int tvo = tm.tt * NV;  // this thread's offset in a thread-private row
@@ -250,6 +287,8 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
       double* exA_w = reinterpret_cast<double*>(sb + lay.exA) + ((t + 1) & 1) * GL;
       const float* exF_r = reinterpret_cast<const float*>(sb + lay.exF) + (t & 1) * GL;
       float* exF_w = reinterpret_cast<float*>(sb + lay.exF) + ((t + 1) & 1) * GL;
+      if (!a0 && t > 0) xwait(X, 0, t & 1);
+      if (write) xarm(X, 0, (t + 1) & 1);
 #pragma unroll
       for (int u = 0; u < U; ++u)
 #pragma unroll
@@ -317,10 +356,17 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
         }
       }
       if (!tm.a_writer) return;
+      const uint32_t bar_l = smem_u32(mbar(X, 0, (t + 1) & 1));
       if (contig) {
         uint32_t r;
         int off;
         tm.a_dest(tm.a_out_index(0, 0), r, off);
+        uint32_t rbar = 0, ra_ = 0, rf_ = 0;
+        if constexpr (CL > 1) {
+          rbar = mapa_u32(bar_l, r);
+          ra_ = mapa_u32(smem_u32(exA_w + off), r);
+          if constexpr (ADJ) rf_ = mapa_u32(smem_u32(exF_w + off), r);
+        }
 #pragma unroll
         for (int v = 0; v < U * BT; v += 2) {
           const double o0 = outs[v / BT][v % BT], o1 = outs[(v + 1) / BT][(v + 1) % BT];
@@ -330,11 +376,8 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
               *reinterpret_cast<float2*>(exF_w + off + v) =
                   make_float2(fos[v / BT][v % BT], fos[(v + 1) / BT][(v + 1) % BT]);
           } else {
-            st_cluster_v2f64(exA_w + off + v, r, o0, o1);
-            if constexpr (ADJ) {
-              team_store<CL>(exF_w, r, off + v, fos[v / BT][v % BT]);
-              team_store<CL>(exF_w, r, off + v + 1, fos[(v + 1) / BT][(v + 1) % BT]);
-            }
+            st_async_v2f64(ra_ + 8u * v, o0, o1, rbar);
+            if constexpr (ADJ) st_async_v2f32(rf_ + 4u * v, fos[v / BT][v % BT], fos[(v + 1) / BT][(v + 1) % BT], rbar);
           }
         }
       } else {
@@ -345,8 +388,14 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
             uint32_t r;
             int off;
             tm.a_dest(tm.a_out_index(u, bb), r, off);
-            team_store_f64<CL>(exA_w, r, off, outs[u][bb]);
-            if constexpr (ADJ) team_store<CL>(exF_w, r, off, fos[u][bb]);
+            if constexpr (CL == 1) {
+              exA_w[off] = outs[u][bb];
+              if constexpr (ADJ) exF_w[off] = fos[u][bb];
+            } else {
+              const uint32_t rbar = mapa_u32(bar_l, r);
+              st_async_f64(mapa_u32(smem_u32(exA_w + off), r), outs[u][bb], rbar);
+              if constexpr (ADJ) st_async_f32(mapa_u32(smem_u32(exF_w + off), r), fos[u][bb], rbar);
+            }
           }
       }
     };
@@ -412,6 +461,7 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
       unsigned char* sb = team_base + static_cast<size_t>(X) * lay.per_seq;
       const double* exA_r = reinterpret_cast<const double*>(sb + lay.exA) + (n & 1) * GL;
       const float* exF_r = reinterpret_cast<const float*>(sb + lay.exF) + (n & 1) * GL;
+      xwait(X, 0, n & 1);
       double av[U][JT];
       uint32_t key = 0xffffffffu;
 #pragma unroll
@@ -561,6 +611,9 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
         }
       }
       // incoming B'_t at the thread's successor groups (q << k) | b
+      if (t < n - 1) xwait(X, setB, t & 1);
+      if (t >= 1) xarm(X, setB, (t + 1) & 1);
+      const uint32_t bar_l = smem_u32(mbar(X, setB, (t + 1) & 1));
       double bv[U][BT];
       float btl[U][BT];
 #pragma unroll
@@ -614,11 +667,18 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
           }
           if (t >= 1 && tm.b_writer) {
             const double out = static_cast<double>(s > 0.f ? lg2f(s) : fbk::kNegLarge) - (r + kd);
+            const float bt_out = (s > 0.f) ? bnum * rcpf(s) : 0.f;
             uint32_t rk;
             int off;
             tm.b_dest(tm.b_out_index(u, jj), rk, off);
-            team_store_f64<CL>(exB_w, rk, off, out);
-            if constexpr (ADJ) team_store<CL>(exBt_w, rk, off, (s > 0.f) ? bnum * rcpf(s) : 0.f);
+            if constexpr (CL == 1) {
+              exB_w[off] = out;
+              if constexpr (ADJ) exBt_w[off] = bt_out;
+            } else {
+              const uint32_t rbar = mapa_u32(bar_l, rk);
+              st_async_f64(mapa_u32(smem_u32(exB_w + off), rk), out, rbar);
+              if constexpr (ADJ) st_async_f32(mapa_u32(smem_u32(exBt_w + off), rk), bt_out, rbar);
+            }
           }
         }
       }
