@@ -24,6 +24,8 @@ namespace bcjr {
 
 constexpr int kStatesPerThread = 16;
 
+constexpr int ilog2_constexpr(int v) { return v <= 1 ? 0 : 1 + ilog2_constexpr(v >> 1); }
+
 __device__ __forceinline__ float ex2f(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

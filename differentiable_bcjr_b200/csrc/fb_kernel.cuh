@@ -164,11 +164,18 @@ template <int K, int CL, bool ADJ, int NSEQ, int NTB>
 __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
   using TL = Tile<K>;
   constexpr int U = TL::U, JT = TL::JT, BT = TL::BT, NV = U * JT;
-  const int L = p.L, k = p.k, n = p.n, C = p.C;
+  // A cluster team fills its cluster exactly (S / 16 = CL * NTB threads), so
+  // the trellis size is a compile-time constant there and every index below
+  // folds to immediates; single-CTA teams take it from the parameters.
+  constexpr int kLog2K = K == 2 ? 1 : K == 4 ? 2 : K == 8 ? 3 : 4;
+  constexpr int kLc = CL > 1 ? ilog2_constexpr(kStatesPerThread * CL * NTB) : 0;
+  const int L = kLc ? kLc : p.L;
+  constexpr int k = kLog2K;
+  const int n = p.n, C = p.C;
   const bool alias = (C == 1);
   const int S = 1 << L;
   const int TS = S / kStatesPerThread;
-  const int NT = static_cast<int>(blockDim.x);
+  const int NT = CL > 1 ? NTB : static_cast<int>(blockDim.x);
   const int tpc = (CL == 1 && TS < NT) ? NT / TS : 1;
   const int team_in_cta = (tpc > 1) ? static_cast<int>(threadIdx.x) / TS : 0;
   Team<K, CL> tm;

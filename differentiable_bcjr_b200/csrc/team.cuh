@@ -15,7 +15,7 @@ struct Team {
   int q0, j0, b0, qloc0;
   bool a_writer, b_writer;
 
-  __device__ void init(int L_, int k_, int team_thread_offset) {
+  __device__ __forceinline__ void init(int L_, int k_, int team_thread_offset) {
     L = L_;
     k = k_;
     S = 1 << L;
