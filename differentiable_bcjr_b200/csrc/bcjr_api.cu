@@ -6,7 +6,7 @@
 #include <cmath>
 #include <cstring>
 
-#include "../../include/bcjr.h"
+#include "bcjr.h"
 #include "bcjr_internal.h"
 
 using bcjr::FBParams;

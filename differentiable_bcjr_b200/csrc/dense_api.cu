@@ -1,5 +1,5 @@
 // dense_api.cu -- dense (fully connected) trellis entry points.
-#include "../../include/bcjr.h"
+#include "bcjr.h"
 #include "bcjr_internal.h"
 
 size_t bcjr_dense_workspace_size_impl(int op, int n_states, int seq_len, int n_seq, const bcjr_options* opt) {
