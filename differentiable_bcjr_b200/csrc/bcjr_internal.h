@@ -109,6 +109,38 @@ struct ViterbiParams {
   int num_slots;
 };
 
+// Dense (fully connected) trellis: 256 states, 32 sequences per CTA.
+constexpr int kDenseStates = 256;
+constexpr int kDenseRows = 32;
+
+struct DenseParams {
+  const float* w;          // [N][n]
+  const float* codebook;   // [S]
+  const float* g;          // [N][n] upstream gradient (backward)
+  const float* what_in;    // [N][n] soft codeword of the forward call (backward; centring)
+  float* w_hat;            // [N][n] (forward)
+  float* marginals;        // [N][n][S] or null (forward)
+  float* log_z;            // [N] or null (forward)
+  float* grad_w;           // [N][n] (backward)
+  float* gc_part;          // [grid][S] per-CTA codebook-gradient partials (backward)
+  const float* P;          // [S][S] exp(Lambda)
+  const float* PT;         // [S][S] its transpose
+  float* ckx;              // per CTA [n][32][S] normalised forward vectors
+  float* ckf;              // per CTA [n][32][S] forward adjoint accumulators (backward)
+  float* mtab;             // per CTA [n][32] emission reference of each step
+  int* status;
+  size_t ck_stride;        // floats per CTA in ckx / ckf
+  size_t mt_stride;        // floats per CTA in mtab
+  float sc2;               // log2(e) / T
+  float two_over_T;
+  int n, N;
+};
+
+// Dense launchers (dense_kernel.cu).
+size_t dense_smem_bytes(bool adjoint);
+cudaError_t dense_geometry(bool adjoint, int n_seq, int* grid);
+cudaError_t launch_dense(const DenseParams& p, const float* lam, bool adjoint, int grid, cudaStream_t s);
+
 // Launchers (bitshift_kernels.cu).  Return a cudaError_t from the launch.
 cudaError_t launch_fb(const FBParams& p, const TeamGeometry& g, bool adjoint, cudaStream_t s);
 cudaError_t launch_viterbi(const ViterbiParams& p, const TeamGeometry& g, cudaStream_t s);

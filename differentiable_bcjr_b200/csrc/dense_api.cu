@@ -1,23 +1,146 @@
-// dense_api.cu -- dense (fully connected) trellis entry points.
+// dense_api.cu -- extern "C" entry points for the dense (fully connected) trellis.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
 #include "bcjr.h"
 #include "bcjr_internal.h"
 
+namespace {
+
+constexpr size_t kHeader = 256;  // int status word + padding
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+struct DenseLayout {
+  size_t P, PT, ckx, ckf, mtab, gc, total, ck_stride, mt_stride;
+};
+
+DenseLayout dense_layout(int grid, int n, bool adjoint) {
+  const size_t S = bcjr::kDenseStates, M = bcjr::kDenseRows;
+  DenseLayout l = {};
+  l.ck_stride = static_cast<size_t>(n) * M * S;
+  l.mt_stride = static_cast<size_t>(n) * M;
+  size_t off = kHeader;
+  l.P = off;
+  off = align_up(off + S * S * sizeof(float));
+  l.PT = off;
+  off = align_up(off + S * S * sizeof(float));
+  l.ckx = off;
+  off = align_up(off + static_cast<size_t>(grid) * l.ck_stride * sizeof(float));
+  l.ckf = off;
+  if (adjoint) off = align_up(off + static_cast<size_t>(grid) * l.ck_stride * sizeof(float));
+  l.mtab = off;
+  off = align_up(off + static_cast<size_t>(grid) * l.mt_stride * sizeof(float));
+  l.gc = off;
+  if (adjoint) off = align_up(off + static_cast<size_t>(grid) * S * sizeof(float));
+  l.total = off;
+  return l;
+}
+
+bcjr_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return BCJR_OK;
+  if (e == cudaErrorNotSupported) return BCJR_ERR_UNSUPPORTED;
+  return BCJR_ERR_CUDA;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// The dense kernels keep every step's forward vector (no recompute schedule).
+bcjr_status check_options(const bcjr_options* opt) {
+  if (!opt) return BCJR_OK;
+  if (opt->checkpoint_interval < 0 || opt->sequences_in_flight < 0 || opt->sequences_in_flight > 1)
+    return BCJR_ERR_INVALID_ARG;
+  if (opt->checkpoint_interval > 1) return BCJR_ERR_UNSUPPORTED;
+  return BCJR_OK;
+}
+
+bcjr_status dense_common(bool adjoint, const float* g, const float* w, const float* c, const float* lam,
+                         const float* what_in, float T, int S, int n, int N, float* w_hat, float* marginals,
+                         float* log_z, float* grad_w, float* grad_c, int accumulate, const bcjr_options* opt,
+                         void* ws, size_t ws_bytes, bcjr_stream_t stream) {
+  if (S < 1 || n < 1 || N < 0 || !(T > 0.f) || !std::isfinite(T)) return BCJR_ERR_INVALID_ARG;
+  bcjr_status st = check_options(opt);
+  if (st != BCJR_OK) return st;
+  if (S != bcjr::kDenseStates) return BCJR_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (N == 0) {
+    if (!adjoint || accumulate) return BCJR_OK;
+    if (!grad_c) return BCJR_ERR_INVALID_ARG;
+    return from_cuda(cudaMemsetAsync(grad_c, 0, S * sizeof(float), s));
+  }
+  if (!w || !c || !lam || !aligned(w, 4) || !aligned(c, 4) || !aligned(lam, 4)) return BCJR_ERR_INVALID_ARG;
+  if (adjoint) {
+    if (!g || !what_in || !grad_w || !grad_c) return BCJR_ERR_INVALID_ARG;
+  } else {
+    if (!w_hat) return BCJR_ERR_INVALID_ARG;
+    if (marginals && !aligned(marginals, 16)) return BCJR_ERR_INVALID_ARG;
+  }
+  if (!ws || !aligned(ws, kAlign)) return BCJR_ERR_WORKSPACE;
+  int grid = 0;
+  if ((st = from_cuda(bcjr::dense_geometry(adjoint, N, &grid))) != BCJR_OK) return st;
+  const DenseLayout lay = dense_layout(grid, n, adjoint);
+  if (ws_bytes < lay.total) return BCJR_ERR_WORKSPACE;
+  char* base = static_cast<char*>(ws);
+  bcjr::DenseParams p = {};
+  p.w = w;
+  p.codebook = c;
+  p.g = g;
+  p.what_in = what_in;
+  p.w_hat = w_hat;
+  p.marginals = marginals;
+  p.log_z = log_z;
+  p.grad_w = grad_w;
+  p.gc_part = reinterpret_cast<float*>(base + lay.gc);
+  p.P = reinterpret_cast<const float*>(base + lay.P);
+  p.PT = reinterpret_cast<const float*>(base + lay.PT);
+  p.ckx = reinterpret_cast<float*>(base + lay.ckx);
+  p.ckf = reinterpret_cast<float*>(base + lay.ckf);
+  p.mtab = reinterpret_cast<float*>(base + lay.mtab);
+  p.status = reinterpret_cast<int*>(base);
+  p.ck_stride = lay.ck_stride;
+  p.mt_stride = lay.mt_stride;
+  p.sc2 = static_cast<float>(1.4426950408889634 / static_cast<double>(T));
+  p.two_over_T = static_cast<float>(2.0 / static_cast<double>(T));
+  p.n = n;
+  p.N = N;
+  if ((st = from_cuda(cudaMemsetAsync(ws, 0, sizeof(int), s))) != BCJR_OK) return st;
+  if ((st = from_cuda(bcjr::launch_dense(p, lam, adjoint, grid, s))) != BCJR_OK) return st;
+  if (adjoint) return from_cuda(bcjr::launch_gradc_reduce(p.gc_part, grid, S, grad_c, accumulate, s));
+  return BCJR_OK;
+}
+
+}  // namespace
+
 size_t bcjr_dense_workspace_size_impl(int op, int n_states, int seq_len, int n_seq, const bcjr_options* opt) {
-  (void)op; (void)n_states; (void)seq_len; (void)n_seq; (void)opt;
-  return 0;
+  if (n_states != bcjr::kDenseStates || seq_len < 1 || n_seq < 0) return 0;
+  if (check_options(opt) != BCJR_OK) return 0;
+  const bool adjoint = (op == BCJR_OP_DENSE_BACKWARD);
+  int grid = 0;
+  if (bcjr::dense_geometry(adjoint, n_seq > 0 ? n_seq : 1, &grid) != cudaSuccess) return 0;
+  return dense_layout(grid, seq_len, adjoint).total;
 }
 
 extern "C" {
 
-bcjr_status bcjr_dense_forward(const float*, const float*, const float*, float, int, int, int, float*, float*,
-                               float*, const bcjr_options*, void*, size_t, bcjr_stream_t) {
-  return BCJR_ERR_UNSUPPORTED;
+bcjr_status bcjr_dense_forward(const float* w, const float* codebook, const float* log_trans, float T,
+                               int n_states, int seq_len, int n_seq, float* w_hat, float* marginals,
+                               float* log_z, const bcjr_options* opt, void* workspace, size_t workspace_bytes,
+                               bcjr_stream_t stream) {
+  return dense_common(false, nullptr, w, codebook, log_trans, nullptr, T, n_states, seq_len, n_seq, w_hat,
+                      marginals, log_z, nullptr, nullptr, 0, opt, workspace, workspace_bytes, stream);
 }
 
-bcjr_status bcjr_dense_backward(const float*, const float*, const float*, const float*, const float*, float, int,
-                                int, int, float*, float*, int, const bcjr_options*, void*, size_t,
-                                bcjr_stream_t) {
-  return BCJR_ERR_UNSUPPORTED;
+bcjr_status bcjr_dense_backward(const float* grad_w_hat, const float* w, const float* codebook,
+                                const float* log_trans, const float* w_hat, float T, int n_states, int seq_len,
+                                int n_seq, float* grad_w, float* grad_codebook, int accumulate_codebook,
+                                const bcjr_options* opt, void* workspace, size_t workspace_bytes,
+                                bcjr_stream_t stream) {
+  return dense_common(true, grad_w_hat, w, codebook, log_trans, w_hat, T, n_states, seq_len, n_seq, nullptr,
+                      nullptr, nullptr, grad_w, grad_codebook, accumulate_codebook, opt, workspace,
+                      workspace_bytes, stream);
 }
 
 }  // extern "C"

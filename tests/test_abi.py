@@ -96,3 +96,35 @@ def test_get_status_rejects_null(lib):
     lib.bcjr_get_status.restype = ctypes.c_int
     lib.bcjr_get_status.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
     assert lib.bcjr_get_status(None, None) == 1
+
+
+class _Opts(ctypes.Structure):
+    _fields_ = [("checkpoint_interval", ctypes.c_int), ("sequences_in_flight", ctypes.c_int),
+                ("reserved", ctypes.c_int * 6)]
+
+
+def test_dense_arguments_are_rejected_on_the_host(lib):
+    INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 3
+    f = lib.bcjr_dense_forward
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_float] + [ctypes.c_int] * 3 + [ctypes.c_void_p] * 3 + \
+        [ctypes.POINTER(_Opts), ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+
+    def call(S=256, n=4, N=2, T=0.5, w=4096, c=8192, lam=12288, what=16384, ws=65536, opt=None):
+        return f(w, c, lam, T, S, n, N, what, None, None, opt, ws, 1 << 20, None)
+
+    assert call(T=0.0) == INVALID
+    assert call(T=float("nan")) == INVALID
+    assert call(n=0) == INVALID
+    assert call(N=-1) == INVALID
+    assert call(S=128) == UNSUPPORTED        # the dense kernels are built for 256 states
+    assert call(w=0) == INVALID
+    assert call(lam=0) == INVALID
+    assert call(what=0) == INVALID
+    assert call(ws=0) == WORKSPACE
+    o = _Opts()
+    o.checkpoint_interval = 4                 # the dense path keeps every step
+    assert call(opt=ctypes.pointer(o)) == UNSUPPORTED
+    o.checkpoint_interval = -1
+    assert call(opt=ctypes.pointer(o)) == INVALID
+    assert call(N=0) == 0                     # nothing to do
