@@ -40,6 +40,9 @@ import bcjr_inputs as I  # noqa: E402
 METRIC = "BCJR fwd+bwd weights/s and state-updates/s at S=2^16,k=2; % of exp-pipe peak"
 WORKLOAD = "proj2048x8192_L16_k2"
 MUFU_OPS_PER_CLK_PER_SM = 16      # ex2/lg2 throughput per SM per clock (compute capability 10.0)
+FP32_FMA_PER_CLK_PER_SM = 128     # float32 fma lanes per SM per clock (compute capability 10.0)
+DENSE_METRIC = "dense BCJR fwd+bwd weights/s at S=256, n=4096, N=4096; % of FP32 peak"
+DENSE_WORKLOAD = "dense_S256"
 ALG_MUFU_PER_STATE_STEP = 4       # one forward and one backward log-sum-exp in each of the two calls
 
 
@@ -55,6 +58,8 @@ def parse():
     ap.add_argument("--seq-in-flight", type=int, default=0, help="sequences per cluster in flight (0 = auto)")
     ap.add_argument("--n-seq", type=int, default=0,
                     help="sequences per GPU (default: the workload's 65536); smaller only for profiling")
+    ap.add_argument("--workload", default="projection", choices=["projection", "dense"],
+                    help="projection: the S=2^16, k=2 headline; dense: the 256-state fully connected trellis")
     return ap.parse_args()
 
 
@@ -384,10 +389,162 @@ def run_gpu(args):
     return 0
 
 
+# --------------------------------------------------------------------------
+# Dense 256-state trellis (the fully connected workload)
+# --------------------------------------------------------------------------
+def dense_oracle_rate(n_seq_sample: int, n_steps: int, T: float):
+    import oracle
+    W = I.WORKLOADS[DENSE_WORKLOAD]
+    S = W["n_states"]
+    c, lam = I.codebook(S), I.log_transition(S)
+    w, g = I.weights(n_seq_sample, n_steps), I.upstream_grad(n_seq_sample, n_steps)
+    cores = len(os.sched_getaffinity(0))
+    threads = min(cores, n_seq_sample)
+    t0 = time.perf_counter()
+    oracle.dense_forward(w, c, lam, T, nthreads=threads)
+    oracle.dense_backward(g, w, c, lam, T, nthreads=threads)
+    dt = time.perf_counter() - t0
+    return n_seq_sample * n_steps / dt, threads, dt
+
+
+def _dense_config(n_gpus, N):
+    W = I.WORKLOADS[DENSE_WORKLOAD]
+    return {"workload": DENSE_WORKLOAD, "n_states": W["n_states"], "seq_len": W["seq_len"], "n_seq_per_gpu": N,
+            "weights_per_gpu": N * W["seq_len"], "T": W["T"][0], "parallelism": f"dp{n_gpus}",
+            "l2": "no flush: each call streams 17-34 GiB of checkpoints, larger than the 126 MB L2"}
+
+
+def run_dense(args):
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    import differentiable_bcjr_b200 as B
+
+    W = I.WORKLOADS[DENSE_WORKLOAD]
+    S, n, N, T = W["n_states"], W["seq_len"], W["n_seq"], W["T"][0]
+    if args.n_seq > 0:
+        N = args.n_seq
+    c_h, lam_h = I.codebook(S), I.log_transition(S)
+    w_h = I.weights(N, n, seed=I.SEED_WEIGHTS + 100 * rank)
+    g_h = I.upstream_grad(N, n, seed=I.SEED_UPSTREAM + 100 * rank)
+    c, lam, w, g = c_h.to(dev), lam_h.to(dev), w_h.to(dev), g_h.to(dev)
+    ws_f, ws_b = B.Workspace(dev), B.Workspace(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(w_in, g_in):
+        w_hat, _, _ = B.bcjr_dense_forward(w_in, c, lam, T, ws=ws_f)
+        gw, gc = B.bcjr_dense_backward(g_in, w_in, c, lam, w_hat, T, ws=ws_b)
+        if world > 1:
+            torch.distributed.all_reduce(gc)
+        return w_hat, gw, gc
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step(w, g)
+    barrier()
+    sampler = ClockSampler(local)
+    sampler.start()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    barrier()
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        w_hat, _, _ = B.bcjr_dense_forward(w, c, lam, T, ws=ws_f)
+        ev[i][1].record(stream)
+        gw, gc = B.bcjr_dense_backward(g, w, c, lam, w_hat, T, ws=ws_b)
+        ev[i][2].record(stream)
+        if world > 1:
+            torch.distributed.all_reduce(gc)
+    barrier()
+    clocks = sampler.stop()
+    fwd_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    bwd_ms = [b.elapsed_time(cc) for _, b, cc in ev]
+    elapsed_ms = ev[0][0].elapsed_time(ev[-1][2])
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / args.steps
+    value = world * N * n / (ms_per_step / 1e3)
+
+    e2e = None
+    if not args.no_e2e:
+        w_pin, g_pin = w_h.pin_memory(), g_h.pin_memory()
+        what_pin, gw_pin = torch.empty_like(w_h).pin_memory(), torch.empty_like(w_h).pin_memory()
+        gc_pin = torch.empty(S).pin_memory()
+        w_d, g_d = torch.empty_like(w), torch.empty_like(g)
+        h2d = (w_pin.numel() + g_pin.numel()) * 4
+        d2h = (what_pin.numel() + gw_pin.numel() + gc_pin.numel()) * 4
+        barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for _ in range(args.steps):
+            w_d.copy_(w_pin, non_blocking=True)
+            g_d.copy_(g_pin, non_blocking=True)
+            w_hat, gw, gc = step(w_d, g_d)
+            what_pin.copy_(w_hat, non_blocking=True)
+            gw_pin.copy_(gw, non_blocking=True)
+            gc_pin.copy_(gc, non_blocking=True)
+        e2.record(stream)
+        barrier()
+        e2e_ms = s2.elapsed_time(e2)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * N * n / (e2e_ms / args.steps / 1e3), "unit": "weights/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps}
+
+    if rank == 0:
+        peaks = load_peaks()
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        max_mhz = float(peaks.get("sm_max_mhz", 1965.0))
+        fp32_peak = 2 * FP32_FMA_PER_CLK_PER_SM * sms * max_mhz * 1e6     # FLOP/s
+        bwd_s = statistics.mean(bwd_ms) / 1e3
+        fwd_s = statistics.mean(fwd_ms) / 1e3
+        flops_b = 2 * 4 * N * n * S * S   # adjoint: two stacked contractions per sweep, two sweeps
+        flops_f = 2 * 2 * N * n * S * S   # forward call: one contraction per sweep, two sweeps
+        line = {
+            "metric": DENSE_METRIC, "value": value, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": _dense_config(world, N),
+            "roofline": {"bound": "alu", "pipe": "FP32 FMA (SIMT)", "achieved": flops_b / bwd_s / 1e12,
+                         "peak": fp32_peak / 1e12, "unit": "TFLOP/s", "frac": flops_b / bwd_s / fp32_peak,
+                         "traffic": None, "kernel": "dense_fb_kernel<adjoint> (bcjr_dense_backward)",
+                         "peak_source": f"2 x {FP32_FMA_PER_CLK_PER_SM} FMA/clk/SM x {sms} SMs x {max_mhz:.0f} MHz"},
+            "forward_call": {"ms": 1e3 * fwd_s, "TFLOP/s": flops_f / fwd_s / 1e12,
+                             "frac": flops_f / fwd_s / fp32_peak},
+            "kernels_ms": {"bcjr_dense_forward": 1e3 * fwd_s, "bcjr_dense_backward": 1e3 * bwd_s},
+            "gpu_launches": 5 * args.steps,
+            "clocks": clocks,
+        }
+        if e2e is not None:
+            line["e2e"] = e2e
+        if world == 1 and not args.no_cpu_baseline:
+            rate, threads, dt = dense_oracle_rate(max(1, min(len(os.sched_getaffinity(0)), 16)), 256, T)
+            line["cpu_baseline"] = {"value": rate, "unit": "weights/s", "cores": threads, "kind": "oracle",
+                                    "sample": f"{threads} sequences x 256 steps of the workload (fwd+bwd), "
+                                              f"{dt:.1f} s of CPU work"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "dense":
+        return run_dense(args)
     return run_gpu(args)
 
 
