@@ -225,12 +225,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
   uint32_t done = 0;
   const long long t0 = clock64();
   while (true) {
+    // The hint lets the thread sleep in hardware until the phase completes
+    // (or 0.1 ms pass) instead of re-issuing the loop.
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(done)
-        : "r"(a), "r"(parity)
+        : "r"(a), "r"(parity), "r"(100000u)
         : "memory");
     if (done) return true;
     if (clock64() - t0 > 4000000000LL) {

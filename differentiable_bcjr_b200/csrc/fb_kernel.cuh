@@ -267,6 +267,7 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
     bool bad;   // an input weight was not finite or out of range
     double K0;  // k (n-1) - log2 Z
     float Dc;   // backward call: E[sum_t g_t (c(s_t) - w_hat_t)]
+    float wq, gq, hq;  // the next step's weight (and upstream gradient, soft codeword), loaded one step ahead
   };
 
   for (int it = 0; it < iters; ++it) {
@@ -280,13 +281,25 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
       sq[x].K0 = 0.0;
       sq[x].Dc = 0.f;
     }
+    // Inputs of sequence X at step t, loaded one step before they are used.
+    auto load_inputs = [&](Seq& c, int t) {
+      const size_t o = static_cast<size_t>(c.seq) * n + t;
+      c.wq = __ldg(p.w + o);
+      if constexpr (ADJ) {
+        c.gq = __ldg(p.g + o);
+        c.hq = __ldg(p.what_in + o);
+      }
+    };
+#pragma unroll
+    for (int x = 0; x < NSEQ; ++x) load_inputs(sq[x], 0);
     fbk::Pipe<CL, NSEQ> pipe;
 
     // Forward step of sequence X at step t: reads A'_t (and F~_t) from the
     // exchange buffers, or from a0/f0 when given; when `write` is set, writes
     // A'_{t+1} (and F~_{t+1}) to the readers' exchange buffers.  Leaves the
     // inputs in a / f.
-    auto forward_step = [&](auto xc, int t, const double* a0, const float* f0, bool write, double* a, float* f) {
+    auto forward_step = [&](auto xc, int t, const double* a0, const float* f0, bool write, double* a, float* f,
+                            float wt, float gt, float gw) {
       constexpr int X = decltype(xc)::value;
       Seq& c = sq[X];
       unsigned char* sb = team_base + static_cast<size_t>(X) * lay.per_seq;
@@ -309,22 +322,8 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
           }
         }
       if (!write) return;
-      const float* wrow = p.w + static_cast<size_t>(c.seq) * n;
-      const float wt = __ldg(wrow + t);
       const double wp = static_cast<double>(wt) * sqsc;
       c.bad |= !(fabs(wp) <= fbk::kMaxScaled);
-      float gt = 0.f, gw = 0.f;
-      if constexpr (ADJ) {
-        gt = __ldg(p.g + static_cast<size_t>(c.seq) * n + t);
-        gw = gt * __ldg(p.what_in + static_cast<size_t>(c.seq) * n + t);
-      }
-      if (t + 1 < n && tm.lane == 0) {
-        asm volatile("prefetch.global.L1 [%0];" ::"l"(wrow + t + 1));
-        if constexpr (ADJ) {
-          asm volatile("prefetch.global.L1 [%0];" ::"l"(p.g + static_cast<size_t>(c.seq) * n + t + 1));
-          asm volatile("prefetch.global.L1 [%0];" ::"l"(p.what_in + static_cast<size_t>(c.seq) * n + t + 1));
-        }
-      }
       double outs[U][BT];
       float fos[U][BT];
 #pragma unroll
@@ -432,9 +431,12 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
     auto alpha_block = [&](auto xc, int t) {
       constexpr int X = decltype(xc)::value;
       const size_t lane_id = static_cast<size_t>(slot) * NSEQ + X;
+      Seq& c = sq[X];
+      const float wt = c.wq, gt = ADJ ? c.gq : 0.f, gw = ADJ ? c.gq * c.hq : 0.f;
+      if (t + 1 < n) load_inputs(c, t + 1);
       double a[NV];
       float f[NV];
-      forward_step(xc, t, nullptr, nullptr, true, a, f);
+      forward_step(xc, t, nullptr, nullptr, true, a, f, wt, gt, gw);
       pipe.before_stores();
       // ---- this step's global stores (outside the barrier's release) ----
       if (C == 1) {
@@ -518,9 +520,12 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
           const double* c64 = p.ck64 + lane_id * p.ck64_stride + static_cast<size_t>(t0 / C) * p.row + tvo;
           const float* cF64 =
               ADJ ? p.ckF64 + lane_id * p.ck64_stride + static_cast<size_t>(t0 / C) * p.row + tvo : nullptr;
+          const size_t o = static_cast<size_t>(sq[X].seq) * n + tp;
+          const float wt = __ldg(p.w + o);
+          const float gt = ADJ ? __ldg(p.g + o) : 0.f, gw = ADJ ? gt * __ldg(p.what_in + o) : 0.f;
           double a[NV];
           float f[NV];
-          forward_step(xc, tp, tp == t0 ? c64 : nullptr, tp == t0 ? cF64 : nullptr, tp < t1, a, f);
+          forward_step(xc, tp, tp == t0 ? c64 : nullptr, tp == t0 ? cF64 : nullptr, tp < t1, a, f, wt, gt, gw);
           store_checkpoint(a, f, p.ck + lane_id * p.ck_stride + static_cast<size_t>(tp - t0) * p.row + tvo,
                            p.ckR + lane_id * p.ckR_stride + static_cast<size_t>(tp - t0) * TS + tm.tt,
                            ADJ ? p.ckF + lane_id * p.ck_stride + static_cast<size_t>(tp - t0) * p.row + tvo : nullptr);
@@ -536,7 +541,6 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
       Seq& c = sq[X];
       unsigned char* sb = team_base + static_cast<size_t>(X) * lay.per_seq;
       const size_t lane_id = static_cast<size_t>(slot) * NSEQ + X;
-      const float* wrow = p.w + static_cast<size_t>(c.seq) * n;
       const double* exB_r = reinterpret_cast<const double*>(sb + lay.exB) + (t & 1) * GL;
       double* exB_w = reinterpret_cast<double*>(sb + lay.exB) + ((t + 1) & 1) * GL;  // (t-1) & 1
       const float* exBt_r = reinterpret_cast<const float*>(sb + lay.exBt) + (t & 1) * GL;
@@ -603,20 +607,10 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
       double rp[NV];
 #pragma unroll
       for (int v = 0; v < NV; ++v) rp[v] = fbk::neg_f2d(ra[v]) + RK;
-      const float wt = __ldg(wrow + t);
+      const float wt = c.wq;
       const double wp = static_cast<double>(wt) * sqsc;
-      float gt = 0.f, gw = 0.f;
-      if constexpr (ADJ) {
-        gt = __ldg(p.g + static_cast<size_t>(c.seq) * n + t);
-        gw = gt * __ldg(p.what_in + static_cast<size_t>(c.seq) * n + t);
-      }
-      if (t >= 1 && tm.lane == 0) {
-        asm volatile("prefetch.global.L1 [%0];" ::"l"(wrow + t - 1));
-        if constexpr (ADJ) {
-          asm volatile("prefetch.global.L1 [%0];" ::"l"(p.g + static_cast<size_t>(c.seq) * n + t - 1));
-          asm volatile("prefetch.global.L1 [%0];" ::"l"(p.what_in + static_cast<size_t>(c.seq) * n + t - 1));
-        }
-      }
+      const float gt = ADJ ? c.gq : 0.f, gw = ADJ ? c.gq * c.hq : 0.f;
+      if (t >= 1) load_inputs(c, t - 1);
       // incoming B'_t at the thread's successor groups (q << k) | b
       if (t < n - 1) xwait(X, setB, t & 1);
       if (t >= 1) xarm(X, setB, (t + 1) & 1);
@@ -720,6 +714,8 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
         cp_async_commit();
       }
     }
+#pragma unroll
+    for (int x = 0; x < NSEQ; ++x) load_inputs(sq[x], n - 1);
     for (int t = n - 1; t >= 0; --t) {
       if (C > 1 && (t == n - 1 || (t + 1) % C == 0)) {
         pipe.drain();
