@@ -633,6 +633,10 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
       float* mrow = (!ADJ && p.marginals && c.act)
                         ? p.marginals + (static_cast<size_t>(c.seq) * n + t) * static_cast<size_t>(S)
                         : nullptr;
+      // The state loop, instantiated with and without the marginal stores so
+      // that a call without marginals carries none of their addressing.
+      auto states = [&](auto with_marginals) {
+      constexpr bool MARG = decltype(with_marginals)::value;
 #pragma unroll
       for (int u = 0; u < U; ++u) {
 #pragma unroll
@@ -648,14 +652,14 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
             s += e;
             if constexpr (!ADJ) {
               acc0 = fmaf(e, cv, acc0);
-              if (mrow) mrow[tm.state(u, jj, bb)] = e + e;
+              if constexpr (MARG) mrow[tm.state(u, jj, bb)] = e + e;
             } else {
               const float eps = fmaf(gt, cv, -gw) + btl[u][bb];
               const float ge = e * eps;
               bnum += ge;
               const float psi = fmaf(e, fbase, ge);  // psi_t(s) / 2
               acc0 = fmaf(psi, cv, acc0);
-              gc[u][jj][bb] += fmaf(gta, e, psi * fmaf(m2T, cv, twa));
+              gc[u][jj][bb] = fmaf(psi, fmaf(m2T, cv, twa), fmaf(gta, e, gc[u][jj][bb]));
             }
           }
           if constexpr (!ADJ) acc1 += s;  // this thread's states only
@@ -682,6 +686,12 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
             }
           }
         }
+      }
+      };
+      if (mrow) {
+        states(std::true_type{});
+      } else {
+        states(std::false_type{});
       }
       const float v0 = group_sum(acc0, tm.width);
       const float v1 = ADJ ? 0.f : group_sum(acc1, tm.width);
