@@ -194,7 +194,8 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
 
   // Codewords of the thread's 16 states: float (for float32 sums) and scaled float64.
   const double sqsc = p.sqsc;
-  float cf[U][JT][BT];
+  static_assert(BT % 2 == 0, "state pairs along b");
+  float2 cf2[U][JT][BT / 2];  // (c(s_b), c(s_b+1)) pairs: the backward sweep works on state pairs
   double cp[U][JT][BT];
   bool bad_cb = false;
 #pragma unroll
@@ -203,19 +204,24 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
     for (int jj = 0; jj < JT; ++jj)
 #pragma unroll
       for (int bb = 0; bb < BT; ++bb) {
-        cf[u][jj][bb] = __ldg(p.codebook + tm.state(u, jj, bb));
-        cp[u][jj][bb] = static_cast<double>(cf[u][jj][bb]) * sqsc;
+        const float cv = __ldg(p.codebook + tm.state(u, jj, bb));
+        if (bb & 1) {
+          cf2[u][jj][bb / 2].y = cv;
+        } else {
+          cf2[u][jj][bb / 2].x = cv;
+        }
+        cp[u][jj][bb] = static_cast<double>(cv) * sqsc;
         bad_cb |= !(fabs(cp[u][jj][bb]) <= fbk::kMaxScaled);
       }
   if (bad_cb) atomicOr(p.status, kDevNonFinite);
-  float gc[U][JT][BT];
+  float2 gc2[U][JT][BT / 2];  // codebook-gradient accumulators (halves), pairs along b
   if constexpr (ADJ) {
 #pragma unroll
     for (int u = 0; u < U; ++u)
 #pragma unroll
       for (int jj = 0; jj < JT; ++jj)
 #pragma unroll
-        for (int bb = 0; bb < BT; ++bb) gc[u][jj][bb] = 0.f;
+        for (int bb = 0; bb < BT / 2; ++bb) gc2[u][jj][bb] = make_float2(0.f, 0.f);
   }
 
   // Exchange mbarriers (cluster teams): per sequence in flight, one per
@@ -348,7 +354,10 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
           for (int jj = 0; jj < JT; ++jj) {
             const float e = ex2f(fbk::neg_d2f(xv[jj] - ref));
             s += e;
-            if constexpr (ADJ) num = fmaf(e, f[u * JT + jj] + fmaf(gt, cf[u][jj][bb], -gw), num);
+            if constexpr (ADJ) {
+              const float cv = (bb & 1) ? cf2[u][jj][bb / 2].y : cf2[u][jj][bb / 2].x;
+              num = fmaf(e, f[u * JT + jj] + fmaf(gt, cv, -gw), num);
+            }
           }
           if constexpr (K >= 8) {
 #pragma unroll
@@ -629,7 +638,10 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
       const float gta = gt * actf;
       const float m2T = -p.two_over_T * actf;
       const float twa = p.two_over_T * wt * actf;
-      float acc0 = 0.f, acc1 = 0.f;
+      const float2 gt2 = make_float2(gt, gt), ngw2 = make_float2(-gw, -gw), gta2 = make_float2(gta, gta);
+      const float2 m2T2 = make_float2(m2T, m2T), twa2 = make_float2(twa, twa);
+      float2 acc02 = make_float2(0.f, 0.f);
+      float acc1 = 0.f;
       float* mrow = (!ADJ && p.marginals && c.act)
                         ? p.marginals + (static_cast<size_t>(c.seq) * n + t) * static_cast<size_t>(S)
                         : nullptr;
@@ -642,26 +654,33 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
 #pragma unroll
         for (int jj = 0; jj < JT; ++jj) {
           const double r = rp[u * JT + jj];
-          float s = 0.f, bnum = 0.f;
           const float fbase = ADJ ? fa[u * JT + jj] - c.Dc : 0.f;
+          // two states per iteration: the float32 arithmetic runs on packed f32x2 instructions
+          float2 s2 = make_float2(0.f, 0.f), bnum2 = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int bb = 0; bb < BT; ++bb) {
-            const float cv = cf[u][jj][bb];
-            const double d = wp - cp[u][jj][bb];
-            const float e = ex2f(fbk::neg_d2f(fma(-d, d, bv[u][bb] + r)));  // gamma_t(s) / 2
-            s += e;
+          for (int bp = 0; bp < BT / 2; ++bp) {
+            const int b0 = 2 * bp, b1 = 2 * bp + 1;
+            const float2 cv = cf2[u][jj][bp];
+            const double d0 = wp - cp[u][jj][b0], d1 = wp - cp[u][jj][b1];
+            const float2 e = make_float2(ex2f(fbk::neg_d2f(fma(-d0, d0, bv[u][b0] + r))),
+                                         ex2f(fbk::neg_d2f(fma(-d1, d1, bv[u][b1] + r))));  // gamma_t / 2
+            s2 = __fadd2_rn(s2, e);
             if constexpr (!ADJ) {
-              acc0 = fmaf(e, cv, acc0);
-              if constexpr (MARG) mrow[tm.state(u, jj, bb)] = e + e;
+              acc02 = __ffma2_rn(e, cv, acc02);
+              if constexpr (MARG) {
+                mrow[tm.state(u, jj, b0)] = e.x + e.x;
+                mrow[tm.state(u, jj, b1)] = e.y + e.y;
+              }
             } else {
-              const float eps = fmaf(gt, cv, -gw) + btl[u][bb];
-              const float ge = e * eps;
-              bnum += ge;
-              const float psi = fmaf(e, fbase, ge);  // psi_t(s) / 2
-              acc0 = fmaf(psi, cv, acc0);
-              gc[u][jj][bb] = fmaf(psi, fmaf(m2T, cv, twa), fmaf(gta, e, gc[u][jj][bb]));
+              const float2 eps = __fadd2_rn(__ffma2_rn(gt2, cv, ngw2), make_float2(btl[u][b0], btl[u][b1]));
+              const float2 ge = __fmul2_rn(e, eps);
+              bnum2 = __fadd2_rn(bnum2, ge);
+              const float2 psi = __ffma2_rn(e, make_float2(fbase, fbase), ge);  // psi_t / 2
+              acc02 = __ffma2_rn(psi, cv, acc02);
+              gc2[u][jj][bp] = __ffma2_rn(psi, __ffma2_rn(m2T2, cv, twa2), __ffma2_rn(gta2, e, gc2[u][jj][bp]));
             }
           }
+          float s = s2.x + s2.y, bnum = bnum2.x + bnum2.y;
           if constexpr (!ADJ) acc1 += s;  // this thread's states only
           if constexpr (K >= 8) {
 #pragma unroll
@@ -693,7 +712,7 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
       } else {
         states(std::false_type{});
       }
-      const float v0 = group_sum(acc0, tm.width);
+      const float v0 = group_sum(acc02.x + acc02.y, tm.width);
       const float v1 = ADJ ? 0.f : group_sum(acc1, tm.width);
       pipe.before_stores();
       if ((tm.lane & (tm.width - 1)) == 0) {
@@ -765,7 +784,8 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
 #pragma unroll
       for (int jj = 0; jj < JT; ++jj)
 #pragma unroll
-        for (int bb = 0; bb < BT; ++bb) gp[tm.state(u, jj, bb)] = 2.f * gc[u][jj][bb];  // gc holds halves
+        for (int bb = 0; bb < BT; ++bb)  // gc holds halves
+          gp[tm.state(u, jj, bb)] = 2.f * ((bb & 1) ? gc2[u][jj][bb / 2].y : gc2[u][jj][bb / 2].x);
   }
   if constexpr (CL > 1) cluster_sync_all();  // no CTA leaves while its shared memory may be addressed
 }
