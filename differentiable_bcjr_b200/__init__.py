@@ -22,7 +22,7 @@ import torch
 __all__ = [
     "LIB_PATH", "lib", "BCJRError", "bcjr_forward", "bcjr_backward", "viterbi_decode",
     "bcjr_dense_forward", "bcjr_dense_backward", "workspace_size", "Workspace",
-    "SoftTrellisQuant", "soft_quantize", "OP_FORWARD", "OP_BACKWARD", "OP_VITERBI",
+    "SoftTrellisQuant", "soft_quantize", "bcjr_forward_static_scratch", "OP_FORWARD", "OP_BACKWARD", "OP_VITERBI",
     "OP_DENSE_FORWARD", "OP_DENSE_BACKWARD", "STATUS",
 ]
 
@@ -184,13 +184,14 @@ def bcjr_forward_static_scratch(w, codebook, T, state_bits, k, w_hat, log_z=None
 
 
 def bcjr_backward(grad_w_hat, w, codebook, w_hat, T, state_bits, k, checkpoint_interval=0, ws=None,
-                  grad_codebook=None, accumulate_codebook=False, sequences_in_flight=0):
-    """VJP of the soft codeword.  Returns (grad_w [N][n], grad_codebook [S])."""
-    _need_cuda(grad_w_hat, w, codebook, w_hat)
+                  grad_codebook=None, accumulate_codebook=False, sequences_in_flight=0, grad_w_out=None):
+    """VJP of the soft codeword.  Returns (grad_w [N][n], grad_codebook [S]); grad_w goes
+    into `grad_w_out` when given."""
+    _need_cuda(grad_w_hat, w, codebook, w_hat, grad_w_out)
     N, n = w.shape
     S = 1 << state_bits
     dev = w.device
-    grad_w = torch.empty((N, n), dtype=torch.float32, device=dev)
+    grad_w = grad_w_out if grad_w_out is not None else torch.empty((N, n), dtype=torch.float32, device=dev)
     if grad_codebook is None:
         grad_codebook = torch.empty((S,), dtype=torch.float32, device=dev)
         accumulate_codebook = False
