@@ -41,6 +41,8 @@ METRIC = "BCJR fwd+bwd weights/s and state-updates/s at S=2^16,k=2; % of exp-pip
 WORKLOAD = "proj2048x8192_L16_k2"
 MUFU_OPS_PER_CLK_PER_SM = 16      # ex2/lg2 throughput per SM per clock (compute capability 10.0)
 FP32_FMA_PER_CLK_PER_SM = 128     # float32 fma lanes per SM per clock (compute capability 10.0)
+FP64_OPS_PER_CLK_PER_SM = 64     # float64 lanes per SM per clock (compute capability 10.0)
+VITERBI_METRIC = "Viterbi hard decode weights/s at S=2^16,k=2 (2048x8192 projection); % of FP64 peak"
 DENSE_METRIC = "dense BCJR fwd+bwd weights/s at S=256, n=4096, N=4096; % of FP32 peak"
 DENSE_WORKLOAD = "dense_S256"
 ALG_MUFU_PER_STATE_STEP = 4       # one forward and one backward log-sum-exp in each of the two calls
@@ -58,8 +60,9 @@ def parse():
     ap.add_argument("--seq-in-flight", type=int, default=0, help="sequences per cluster in flight (0 = auto)")
     ap.add_argument("--n-seq", type=int, default=0,
                     help="sequences per GPU (default: the workload's 65536); smaller only for profiling")
-    ap.add_argument("--workload", default="projection", choices=["projection", "dense"],
-                    help="projection: the S=2^16, k=2 headline; dense: the 256-state fully connected trellis")
+    ap.add_argument("--workload", default="projection", choices=["projection", "dense", "viterbi"],
+                    help="projection: the S=2^16, k=2 headline; dense: the 256-state fully connected trellis; "
+                         "viterbi: hard decode of the projection")
     return ap.parse_args()
 
 
@@ -539,12 +542,128 @@ def run_dense(args):
     return 0
 
 
+# --------------------------------------------------------------------------
+# Hard decode of the projection (Viterbi, float64 max-sum)
+# --------------------------------------------------------------------------
+def run_viterbi(args):
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    import differentiable_bcjr_b200 as B
+
+    W = I.WORKLOADS[WORKLOAD]
+    L, k, n, N = W["state_bits"], W["k"], W["seq_len"], W["n_seq"]
+    if args.n_seq > 0:
+        N = args.n_seq
+    S = 1 << L
+    c_h = I.codebook(S)
+    w_h = I.weights(N, n, seed=I.SEED_WEIGHTS + 100 * rank)
+    c, w = c_h.to(dev), w_h.to(dev)
+    ws = B.Workspace(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        B.viterbi_decode(w, c, L, k, ws=ws)
+    barrier()
+    sampler = ClockSampler(local)
+    sampler.start()
+    s0, e0 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    s0.record(stream)
+    for _ in range(args.steps):
+        states, w_hard = B.viterbi_decode(w, c, L, k, ws=ws)
+    e0.record(stream)
+    barrier()
+    clocks = sampler.stop()
+    ms = s0.elapsed_time(e0)
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = world * N * n / (ms_per_step / 1e3)
+
+    e2e = None
+    if not args.no_e2e:
+        w_pin = w_h.pin_memory()
+        st_pin = torch.empty((N, n), dtype=torch.int32).pin_memory()
+        wh_pin = torch.empty_like(w_h).pin_memory()
+        w_d = torch.empty_like(w)
+        barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for _ in range(args.steps):
+            w_d.copy_(w_pin, non_blocking=True)
+            states, w_hard = B.viterbi_decode(w_d, c, L, k, ws=ws)
+            st_pin.copy_(states, non_blocking=True)
+            wh_pin.copy_(w_hard, non_blocking=True)
+        e2.record(stream)
+        barrier()
+        e2e_ms = s2.elapsed_time(e2)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": world * N * n / (e2e_ms / args.steps / 1e3), "unit": "weights/s",
+               "h2d_bytes_per_step": w_pin.numel() * 4, "d2h_bytes_per_step": st_pin.numel() * 4 + wh_pin.numel() * 4,
+               "ms_per_step": e2e_ms / args.steps}
+
+    if rank == 0:
+        peaks = load_peaks()
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        max_mhz = float(peaks.get("sm_max_mhz", 1965.0))
+        fp64_peak = FP64_OPS_PER_CLK_PER_SM * sms * max_mhz * 1e6
+        ops = 3 * N * n * S  # subtract, square, add per state-step (float64)
+        line = {
+            "metric": VITERBI_METRIC, "value": value, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": dict(_config(world, 1, N), workload=f"{WORKLOAD} (hard decode)"),
+            "roofline": {"bound": "alu", "pipe": "FP64", "achieved": ops / (ms_per_step / 1e3) / 1e12,
+                         "peak": fp64_peak / 1e12, "unit": "T fp64 op/s",
+                         "frac": ops / (ms_per_step / 1e3) / fp64_peak, "traffic": None,
+                         "kernel": "viterbi_kernel (viterbi_decode)",
+                         "peak_source": f"{FP64_OPS_PER_CLK_PER_SM} fp64 lanes/clk/SM x {sms} SMs x {max_mhz:.0f} MHz"},
+            "kernels_ms": {"viterbi_decode": ms_per_step},
+            "gpu_launches": args.steps,
+            "clocks": clocks,
+        }
+        if e2e is not None:
+            line["e2e"] = e2e
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+            cores = len(os.sched_getaffinity(0))
+            sample = max(1, min(cores, 16))
+            wq = I.weights(sample, n)
+            t0 = time.perf_counter()
+            oracle.viterbi(wq, c_h, L, k, nthreads=min(cores, sample))
+            dt = time.perf_counter() - t0
+            line["cpu_baseline"] = {"value": sample * n / dt, "unit": "weights/s", "cores": min(cores, sample),
+                                    "kind": "oracle", "sample": f"{sample} whole sequences, {dt:.1f} s of CPU work"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
     if args.workload == "dense":
         return run_dense(args)
+    if args.workload == "viterbi":
+        return run_viterbi(args)
     return run_gpu(args)
 
 

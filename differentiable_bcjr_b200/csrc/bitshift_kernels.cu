@@ -12,176 +12,13 @@
 #include "bcjr_device.cuh"
 #include "bcjr_internal.h"
 #include "team.cuh"
+#include "viterbi_kernel.cuh"
 
 namespace bcjr {
 
 namespace {
 constexpr unsigned kFull = 0xffffffffu;
 }  // namespace
-
-// ---------------------------------------------------------------------------
-// Hard decode: max-sum over -(w - c)^2 in float64, each difference, square and
-// sum rounded separately, ties to the lowest predecessor index and the lowest
-// final state ("BCJR-QAT", technical summary: T -> 0 recovers the hard Viterbi
-// output).  Backpointers (k bits, stored as bytes) go to the workspace; one
-// thread of the team walks them back.
-// ---------------------------------------------------------------------------
-template <int K, int CL, int NTB>
-__global__ void __launch_bounds__(NTB, 1) viterbi_kernel(const ViterbiParams p) {
-  using TL = Tile<K>;
-  constexpr int U = TL::U, JT = TL::JT, BT = TL::BT;
-  const int L = p.L, k = p.k, n = p.n;
-  const int S = 1 << L;
-  const int TS = S / kStatesPerThread;
-  const int tpc = (CL == 1 && TS < static_cast<int>(blockDim.x)) ? static_cast<int>(blockDim.x) / TS : 1;
-  const int team_in_cta = (tpc > 1) ? static_cast<int>(threadIdx.x) / TS : 0;
-  Team<K, CL> tm;
-  tm.init(L, k, team_in_cta * TS);
-  const int slot = (CL > 1) ? static_cast<int>(blockIdx.x) / CL : static_cast<int>(blockIdx.x) * tpc + team_in_cta;
-  const int G = tm.G, GL = tm.GL;
-
-  extern __shared__ __align__(16) double smemd[];
-  double* base = smemd + team_in_cta * (2 * static_cast<size_t>(GL) + 2 * 128);
-  double* bufV = base;                 // [2][GL]
-  double* redv = bufV + 2 * GL;        // [128]
-  int* reds = reinterpret_cast<int*>(redv + 128);  // [128]
-
-  float cb[U][JT][BT];
-#pragma unroll
-  for (int u = 0; u < U; ++u)
-#pragma unroll
-    for (int jj = 0; jj < JT; ++jj)
-#pragma unroll
-      for (int bb = 0; bb < BT; ++bb) cb[u][jj][bb] = __ldg(p.codebook + tm.state(u, jj, bb));
-
-  uint8_t* bp = p.bp + static_cast<size_t>(slot) * p.bp_stride;
-  // Every CTA of the cluster must be running before any of them writes into
-  // another's shared memory.
-  if constexpr (CL > 1) cluster_sync_all();
-  const int iters = (p.N + p.num_slots - 1) / p.num_slots;
-  for (int it = 0; it < iters; ++it) {
-    const int seq_raw = slot + it * p.num_slots;
-    const bool active = seq_raw < p.N;
-    const int seq = active ? seq_raw : p.N - 1;
-    const float* wseq = p.w + static_cast<size_t>(seq) * n;
-    double best[U][BT];
-    int bj[U][BT];
-    for (int t = 0; t < n; ++t) {
-      const double wt = static_cast<double>(__ldg(wseq + t));
-      double a[U][JT];
-#pragma unroll
-      for (int u = 0; u < U; ++u)
-#pragma unroll
-        for (int jj = 0; jj < JT; ++jj)
-          a[u][jj] = (t == 0) ? 0.0 : bufV[(t & 1) * GL + tm.a_read_off(u, jj)];
-#pragma unroll
-      for (int u = 0; u < U; ++u)
-#pragma unroll
-        for (int bb = 0; bb < BT; ++bb) {
-          double bv = -DBL_MAX;
-          int bjj = 0;
-#pragma unroll
-          for (int jj = 0; jj < JT; ++jj) {
-            const double d = __dsub_rn(wt, static_cast<double>(cb[u][jj][bb]));
-            const double v = __dadd_rn(a[u][jj], -__dmul_rn(d, d));
-            if (jj == 0 || v > bv) {
-              bv = v;
-              bjj = tm.j0 + jj;
-            }
-          }
-          if constexpr (K >= 8) {
-#pragma unroll
-            for (int o = TL::NBT; o < TL::TPU; o <<= 1) {
-              const double ov = __shfl_xor_sync(kFull, bv, o);
-              const int oj = __shfl_xor_sync(kFull, bjj, o);
-              if (ov > bv || (ov == bv && oj < bjj)) {
-                bv = ov;
-                bjj = oj;
-              }
-            }
-          }
-          best[u][bb] = bv;
-          bj[u][bb] = bjj;
-        }
-      if (t + 1 < n && tm.a_writer) {
-        uint8_t* brow = bp + static_cast<size_t>(t + 1) * G;
-#pragma unroll
-        for (int u = 0; u < U; ++u)
-#pragma unroll
-          for (int bb = 0; bb < BT; ++bb) {
-            const int gi = tm.a_out_index(u, bb);
-            uint32_t r;
-            int off;
-            tm.a_dest(gi, r, off);
-            team_store_f64<CL>(bufV + ((t + 1) & 1) * GL, r, off, best[u][bb]);
-            brow[gi] = static_cast<uint8_t>(bj[u][bb]);
-          }
-      }
-      team_sync<CL>();
-    }
-    // End state: the largest final metric, lowest state on ties.
-    double vb = -DBL_MAX;
-    int sb = S;  // S marks "no candidate"; every reduction below keeps a valid state when one exists
-    if (tm.a_writer) {
-#pragma unroll
-      for (int u = 0; u < U; ++u)
-#pragma unroll
-        for (int bb = 0; bb < BT; ++bb) {
-          const int st = (bj[u][bb] << (L - k)) | tm.a_out_index(u, bb);
-          if (sb == S || best[u][bb] > vb || (best[u][bb] == vb && st < sb)) {
-            vb = best[u][bb];
-            sb = st;
-          }
-        }
-    }
-    for (int o = tm.width >> 1; o > 0; o >>= 1) {
-      const double ov = __shfl_xor_sync(kFull, vb, o);
-      const int os = __shfl_xor_sync(kFull, sb, o);
-      if (os != S && (sb == S || ov > vb || (ov == vb && os < sb))) {
-        vb = ov;
-        sb = os;
-      }
-    }
-    if (tm.TS > 32) {
-      if (tm.lane == 0) {
-        for (int r = 0; r < CL; ++r) {
-          team_store_f64<CL>(redv, r, tm.warp_in_team, vb);
-          team_store_u32<CL>(reinterpret_cast<uint32_t*>(reds), r, tm.warp_in_team, static_cast<uint32_t>(sb));
-        }
-      }
-      team_sync<CL>();
-      vb = -DBL_MAX;
-      sb = S;
-      for (int i = 0; i < tm.wpt; ++i) {
-        const double ov = redv[i];
-        const int os = reds[i];
-        if (os != S && (sb == S || ov > vb || (ov == vb && os < sb))) {
-          vb = ov;
-          sb = os;
-        }
-      }
-    }
-    // Non-finite metrics (NaN inputs) can leave no comparable candidate: keep the walk in range.
-    if (sb < 0 || sb >= S) sb = 0;
-    if (tm.tt == 0 && active) {
-      if (!isfinite(vb)) atomicOr(p.status, kDevNonFinite);
-      if (p.metric) p.metric[seq] = vb;
-      int s = sb;
-      int32_t* st = p.states + static_cast<size_t>(seq) * n;
-      float* wh = p.w_hard ? p.w_hard + static_cast<size_t>(seq) * n : nullptr;
-      for (int t = n - 1; t >= 0; --t) {
-        st[t] = s;
-        if (wh) wh[t] = __ldg(p.codebook + s);
-        if (t >= 1) {
-          const int j = bp[static_cast<size_t>(t) * G + (s >> k)];
-          s = (j << (L - k)) | (s >> k);
-        }
-      }
-    }
-    team_sync<CL>();
-  }
-  if constexpr (CL > 1) cluster_sync_all();
-}
 
 // grad_codebook[s] (+)= sum over teams of the per-team partials, in team order.
 __global__ void gradc_reduce_kernel(const float* __restrict__ part, int num_slots, int S,
@@ -207,7 +44,8 @@ const void* fb_adj_kernel_k4(int cluster, int nseq);
 
 namespace {
 
-constexpr int kFBBlockThreads = 512;  // 16 states per thread, <= 128 registers per thread
+constexpr int kFBBlockThreads = 512;   // 16 states per thread, <= 128 registers per thread
+constexpr int kVitBlockThreads = 512;
 
 const void* pick_fb(bool adjoint, int k, int cl, int nseq) {
   switch (k) {
@@ -220,12 +58,12 @@ const void* pick_fb(bool adjoint, int k, int cl, int nseq) {
 }
 
 const void* pick_viterbi(int k, int cl) {
-#define BCJR_V_CASE(KK, CC) \
-  if (k == KK && cl == CC) return reinterpret_cast<const void*>(&viterbi_kernel<(1 << KK), CC, 1024>);
-  BCJR_V_CASE(1, 1) BCJR_V_CASE(1, 2) BCJR_V_CASE(1, 4)
-  BCJR_V_CASE(2, 1) BCJR_V_CASE(2, 2) BCJR_V_CASE(2, 4)
-  BCJR_V_CASE(3, 1) BCJR_V_CASE(3, 2) BCJR_V_CASE(3, 4)
-  BCJR_V_CASE(4, 1) BCJR_V_CASE(4, 2) BCJR_V_CASE(4, 4)
+#define BCJR_V_CASE(KK, CC, NS) \
+  if (k == KK && cl == CC) return reinterpret_cast<const void*>(&viterbi_kernel<(1 << KK), CC, NS, kVitBlockThreads>);
+  BCJR_V_CASE(1, 1, 1) BCJR_V_CASE(1, 2, 2) BCJR_V_CASE(1, 4, 2) BCJR_V_CASE(1, 8, 2)
+  BCJR_V_CASE(2, 1, 1) BCJR_V_CASE(2, 2, 2) BCJR_V_CASE(2, 4, 2) BCJR_V_CASE(2, 8, 2)
+  BCJR_V_CASE(3, 1, 1) BCJR_V_CASE(3, 2, 2) BCJR_V_CASE(3, 4, 2) BCJR_V_CASE(3, 8, 2)
+  BCJR_V_CASE(4, 1, 1) BCJR_V_CASE(4, 2, 2) BCJR_V_CASE(4, 4, 2) BCJR_V_CASE(4, 8, 2)
 #undef BCJR_V_CASE
   return nullptr;
 }
@@ -400,11 +238,13 @@ cudaError_t viterbi_geometry(int L, int k, int n_seq, TeamGeometry* g) {
     }
   }
   TeamGeometry gg = {};
-  base_geometry(L, 1024, &gg);
+  base_geometry(L, kVitBlockThreads, &gg);
   const int GL = ((1 << L) >> k) / gg.cluster;
-  gg.smem_bytes = (2 * static_cast<size_t>(GL) + 2 * 128) * sizeof(double) * gg.teams_per_cta;
+  gg.nseq = gg.cluster > 1 ? 2 : 1;  // the same as the kernel instantiations
+  gg.smem_bytes = (static_cast<size_t>(gg.nseq) * (2 * GL + 2) + 192) * sizeof(double) * gg.teams_per_cta;
+  if (gg.smem_bytes > static_cast<size_t>(max_optin_smem())) e = cudaErrorNotSupported;
   const void* fn = pick_viterbi(k, gg.cluster);
-  e = fn ? persistent_grid(fn, n_seq, &gg) : cudaErrorNotSupported;
+  if (e == cudaSuccess) e = fn ? persistent_grid(fn, (n_seq + gg.nseq - 1) / gg.nseq, &gg) : cudaErrorNotSupported;
   if (e == cudaSuccess || e == cudaErrorNotSupported) {
     std::lock_guard<std::mutex> lk(g_geo_mu);
     g_geo_cache[key] = {e, gg};
