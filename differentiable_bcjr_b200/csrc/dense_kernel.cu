@@ -26,7 +26,9 @@
 // row-broadcast reads and the transposing writes are conflict-free) and P or
 // P^T streams through a double-buffered shared-memory window of 32 rows with
 // cp.async.  A thread holds RQ sequences x 8 states (states 4l..4l+3 and
-// 128+4l..128+4l+3 of lane l), so state sums are warp shuffles.
+// 128+4l..128+4l+3 of lane l), so state sums are warp shuffles; the
+// contraction runs on packed f32x2 fused multiply-adds over state pairs (each
+// lane rounds exactly as a scalar fma would).
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -155,7 +157,8 @@ __global__ void __launch_bounds__(dense::Cfg<ADJ>::THREADS, 1) dense_fb_kernel(c
         const int s = kc * kKC + kk;
         const float4 b0 = *reinterpret_cast<const float4*>(Pb + kk * kS + 4 * lane);
         const float4 b1 = *reinterpret_cast<const float4*>(Pb + kk * kS + 128 + 4 * lane);
-        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        const float2 bv2[4] = {make_float2(b0.x, b0.y), make_float2(b0.z, b0.w), make_float2(b1.x, b1.y),
+                               make_float2(b1.z, b1.w)};
 #pragma unroll
         for (int g = 0; g < RQ / 4; ++g) {
           const int q = RQ * wp + 4 * g;
@@ -164,14 +167,24 @@ __global__ void __launch_bounds__(dense::Cfg<ADJ>::THREADS, 1) dense_fb_kernel(c
 #pragma unroll
           for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc1[4 * g + i][j] = fmaf(av[i], bv[j], acc1[4 * g + i][j]);
+            for (int j = 0; j < 4; ++j) {
+              float2 c2 = make_float2(acc1[4 * g + i][2 * j], acc1[4 * g + i][2 * j + 1]);
+              c2 = __ffma2_rn(make_float2(av[i], av[i]), bv2[j], c2);
+              acc1[4 * g + i][2 * j] = c2.x;
+              acc1[4 * g + i][2 * j + 1] = c2.y;
+            }
           if constexpr (ADJ) {
             const float4 a2 = *reinterpret_cast<const float4*>(A2 + a_index(s, q));
             const float av2[4] = {a2.x, a2.y, a2.z, a2.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
-              for (int j = 0; j < 8; ++j) acc2[4 * g + i][j] = fmaf(av2[i], bv[j], acc2[4 * g + i][j]);
+              for (int j = 0; j < 4; ++j) {
+                float2 c2 = make_float2(acc2[4 * g + i][2 * j], acc2[4 * g + i][2 * j + 1]);
+                c2 = __ffma2_rn(make_float2(av2[i], av2[i]), bv2[j], c2);
+                acc2[4 * g + i][2 * j] = c2.x;
+                acc2[4 * g + i][2 * j + 1] = c2.y;
+              }
           }
         }
       }
