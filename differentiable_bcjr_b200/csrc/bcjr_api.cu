@@ -93,7 +93,7 @@ ViterbiLayout viterbi_layout(const TeamGeometry& g, int L, int k, int n) {
   const size_t G = static_cast<size_t>(1) << (L - k);
   l.bp_stride = static_cast<size_t>(n) * G;
   l.bp = kHeaderBytes;
-  l.total = align_up(l.bp + static_cast<size_t>(g.num_slots) * g.nseq * l.bp_stride);
+  l.total = align_up(l.bp + static_cast<size_t>(g.num_slots) * g.nseq * 2 * l.bp_stride);  // two buffers per lane
   return l;
 }
 

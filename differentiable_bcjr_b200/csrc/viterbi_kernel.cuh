@@ -12,8 +12,10 @@
 // reader CTA's double-buffered shared memory and are awaited on mbarriers; the
 // relaxed split cluster barrier orders buffer reuse, and two sequences are in
 // flight per cluster.  Backpointers (the argmax j, one byte per group and
-// step, packed into one store per thread-step) go to the workspace; one
-// thread of the team walks them back.
+// step, packed into one store per thread-step) go to a double-buffered
+// workspace area; one thread per sequence walks them back during the forward
+// steps of the next sequences, one walk step per forward step, so that the
+// latency of each dependent load hides behind a step of max-sum work.
 #pragma once
 #include <cfloat>
 #include <cmath>
@@ -97,6 +99,32 @@ __global__ void __launch_bounds__(NTB, 1) viterbi_kernel(const ViterbiParams p) 
 
   const int nsl = p.num_slots;
   const int iters = (p.N + nsl * NSEQ - 1) / (nsl * NSEQ);
+  // Backpointers of sequence slot X in iteration `it` (two buffers, by the parity of it).
+  auto bp_buf = [&](int X, int it_) {
+    return p.bp + ((static_cast<size_t>(slot) * NSEQ + X) * 2 + (it_ & 1)) * p.bp_stride;
+  };
+  // The walker of sequence slot X: lane 0 of warp X of the team.
+  auto is_walker = [&](int X) { return tm.tt == 32 * X; };
+  // Walk state of the previous sequence in each slot (kept by its walker).
+  int wk_s[NSEQ], wk_j[NSEQ], wk_seq[NSEQ];
+  bool wk_act[NSEQ];
+  const uint8_t* wk_bp[NSEQ];
+#pragma unroll
+  for (int x = 0; x < NSEQ; ++x) {
+    wk_s[x] = 0;
+    wk_j[x] = 0;
+    wk_seq[x] = 0;
+    wk_act[x] = false;
+    wk_bp[x] = nullptr;
+  }
+  // One walk step at time index ti (counting down from n-1); the backpointer
+  // loaded here is consumed by the next step.
+  auto walk_step = [&](int x, int ti) {
+    if (ti < n - 1) wk_s[x] = (wk_j[x] << (L - k)) | (wk_s[x] >> k);
+    p.states[static_cast<size_t>(wk_seq[x]) * n + ti] = wk_s[x];
+    if (p.w_hard) p.w_hard[static_cast<size_t>(wk_seq[x]) * n + ti] = __ldg(p.codebook + wk_s[x]);
+    if (ti >= 1) wk_j[x] = wk_bp[x][static_cast<size_t>(ti) * G + (wk_s[x] >> k)];
+  };
   for (int it = 0; it < iters; ++it) {
     int seq[NSEQ];
     bool act[NSEQ];
@@ -191,10 +219,10 @@ __global__ void __launch_bounds__(NTB, 1) viterbi_kernel(const ViterbiParams p) 
         }
       }
       pipe.before_stores();
+      if (wk_act[X] && is_walker(X)) walk_step(X, n - 1 - t);  // previous sequence of this slot
       if (write && tm.a_writer) {
         // the thread's groups a_out_index(u, bb) are NB consecutive bytes
-        uint8_t* brow = p.bp + (static_cast<size_t>(slot) * NSEQ + X) * p.bp_stride + static_cast<size_t>(t + 1) * G +
-                        tm.a_out_index(0, 0);
+        uint8_t* brow = bp_buf(X, it) + static_cast<size_t>(t + 1) * G + tm.a_out_index(0, 0);
         uint64_t packed = 0;
 #pragma unroll
         for (int v = 0; v < NB; ++v)
@@ -265,29 +293,27 @@ __global__ void __launch_bounds__(NTB, 1) viterbi_kernel(const ViterbiParams p) 
       send[x] = sb;
       vend[x] = vb;
     }
-    // Every thread's backpointer stores are visible to the walker after this barrier.
+    // Every thread's backpointer stores are visible to the walkers after this
+    // barrier; they walk this iteration's sequences during the next one.
     team_sync<CL>();
-    if (tm.tt == 0) {
 #pragma unroll
-      for (int x = 0; x < NSEQ; ++x) {
-        if (!act[x]) continue;
+    for (int x = 0; x < NSEQ; ++x) {
+      if (tm.tt == 0 && act[x]) {
         if (!isfinite(vend[x])) atomicOr(p.status, kDevNonFinite);
         if (p.metric) p.metric[seq[x]] = vend[x];
-        const uint8_t* bp = p.bp + (static_cast<size_t>(slot) * NSEQ + x) * p.bp_stride;
-        int s = send[x];
-        int32_t* st = p.states + static_cast<size_t>(seq[x]) * n;
-        float* wh = p.w_hard ? p.w_hard + static_cast<size_t>(seq[x]) * n : nullptr;
-        for (int t = n - 1; t >= 0; --t) {
-          st[t] = s;
-          if (wh) wh[t] = __ldg(p.codebook + s);
-          if (t >= 1) {
-            const int j = bp[static_cast<size_t>(t) * G + (s >> k)];
-            s = (j << (L - k)) | (s >> k);
-          }
-        }
       }
+      wk_s[x] = send[x];
+      wk_seq[x] = seq[x];
+      wk_act[x] = act[x];
+      wk_bp[x] = bp_buf(x, it);
     }
-    team_sync<CL>();  // the backpointers are rewritten by the next sequences
+  }
+  // The sequences of the last iteration are walked back here.
+#pragma unroll
+  for (int x = 0; x < NSEQ; ++x) {
+    if (wk_act[x] && is_walker(x)) {
+      for (int ti = n - 1; ti >= 0; --ti) walk_step(x, ti);
+    }
   }
   if constexpr (CL > 1) cluster_sync_all();  // no CTA leaves while its shared memory may be addressed
 }
