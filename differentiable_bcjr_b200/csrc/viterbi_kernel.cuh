@@ -136,11 +136,15 @@ __global__ void __launch_bounds__(NTB, 1) viterbi_kernel(const ViterbiParams p) 
     }
     double best[NSEQ][U][BT];
     int bj[NSEQ][U][BT];
+    float wnext[NSEQ];  // each step's weight, loaded one step ahead
+#pragma unroll
+    for (int x = 0; x < NSEQ; ++x) wnext[x] = __ldg(p.w + static_cast<size_t>(seq[x]) * n);
     fbk::Pipe<CL, NSEQ> pipe;
 
     auto block = [&](auto xc, int t) {
       constexpr int X = decltype(xc)::value;
-      const double wt = static_cast<double>(__ldg(p.w + static_cast<size_t>(seq[X]) * n + t));
+      const double wt = static_cast<double>(wnext[X]);
+      if (t + 1 < n) wnext[X] = __ldg(p.w + static_cast<size_t>(seq[X]) * n + t + 1);
       if (t > 0) xwait(X, t & 1);
       const bool write = t + 1 < n;
       if (write) xarm(X, (t + 1) & 1);
