@@ -57,7 +57,6 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--checkpoint-interval", type=int, default=1)
-    ap.add_argument("--seq-in-flight", type=int, default=0, help="sequences per cluster in flight (0 = auto)")
     ap.add_argument("--n-seq", type=int, default=0,
                     help="sequences per GPU (default: the workload's 65536); smaller only for profiling")
     ap.add_argument("--workload", default="projection", choices=["projection", "dense", "viterbi"],
@@ -258,11 +257,9 @@ def run_gpu(args):
 
     def step(i, w_in, g_in, what_out):
         T = temps[i % len(temps)]
-        B.bcjr_forward(w_in, c, T, L, k, checkpoint_interval=C, ws=ws_f, out=what_out,
-                       sequences_in_flight=args.seq_in_flight)
+        B.bcjr_forward(w_in, c, T, L, k, checkpoint_interval=C, ws=ws_f, out=what_out)
         gw, gc = B.bcjr_backward(g_in, w_in, c, what_out, T, L, k, checkpoint_interval=C, ws=ws_b,
-                                 grad_codebook=grad_c, accumulate_codebook=False,
-                                 sequences_in_flight=args.seq_in_flight)
+                                 grad_codebook=grad_c, accumulate_codebook=False)
         if world > 1:
             torch.distributed.all_reduce(gc)
         return gw, gc
@@ -288,12 +285,10 @@ def run_gpu(args):
     for i in range(args.steps):
         T = temps[i % len(temps)]
         ev[i][0].record(stream)
-        B.bcjr_forward(w, c, T, L, k, checkpoint_interval=C, ws=ws_f, out=w_hat,
-                       sequences_in_flight=args.seq_in_flight)
+        B.bcjr_forward(w, c, T, L, k, checkpoint_interval=C, ws=ws_f, out=w_hat)
         ev[i][1].record(stream)
         gw, gc = B.bcjr_backward(g, w, c, w_hat, T, L, k, checkpoint_interval=C, ws=ws_b,
-                                 grad_codebook=grad_c, accumulate_codebook=False,
-                                 sequences_in_flight=args.seq_in_flight)
+                                 grad_codebook=grad_c, accumulate_codebook=False)
         ev[i][2].record(stream)
         if world > 1:
             torch.distributed.all_reduce(gc)

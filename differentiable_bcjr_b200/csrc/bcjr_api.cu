@@ -158,7 +158,7 @@ static bcjr_status fb_common(bool adjoint, const float* grad_w_hat, const float*
   bcjr_status st = check_trellis(L, k);
   if (st != BCJR_OK) return st;
   if (n < 1 || N < 0 || !(T > 0.f) || !std::isfinite(T)) return BCJR_ERR_INVALID_ARG;
-  if (opt && (opt->checkpoint_interval < 0 || opt->sequences_in_flight < 0 || opt->sequences_in_flight > 1))
+  if (opt && (opt->checkpoint_interval < 0 || opt->sequences_in_flight != 0))
     return BCJR_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int S = 1 << L;

@@ -51,7 +51,7 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 // The dense kernels keep every step's forward vector (no recompute schedule).
 bcjr_status check_options(const bcjr_options* opt) {
   if (!opt) return BCJR_OK;
-  if (opt->checkpoint_interval < 0 || opt->sequences_in_flight < 0 || opt->sequences_in_flight > 1)
+  if (opt->checkpoint_interval < 0 || opt->sequences_in_flight != 0)
     return BCJR_ERR_INVALID_ARG;
   if (opt->checkpoint_interval > 1) return BCJR_ERR_UNSUPPORTED;
   return BCJR_OK;

@@ -59,8 +59,9 @@ typedef struct {
   /* Keep the forward group vector every C steps and recompute the others
    * during the backward sweep; 0 selects C = 1 (keep every step). */
   int checkpoint_interval;
-  /* Sequences a thread-block cluster keeps in flight: 0 = automatic, 1.
-   * (Other values are rejected; the interleaved schedule is not offered.) */
+  /* Sequences a team keeps in flight; must be 0 (automatic: two per
+   * thread-block cluster when k >= 2, so that one sequence's step hides the
+   * other's barrier, and one otherwise).  Other values are rejected. */
   int sequences_in_flight;
   int reserved[6]; /* set to zero */
 } bcjr_options;
@@ -154,7 +155,9 @@ bcjr_status viterbi_decode(const float* w, const float* codebook, int state_bits
  * (a 1D Ising-like chain).  Path log-weight sum_t phi_t(s_t) +
  * sum_{t>=1} log_trans[s_{t-1}][s_t]; log_trans is [n_states][n_states],
  * row = source state.  Same outputs and conventions as the bitshift calls.
- * Supported: n_states = 256.
+ * Supported: n_states = 256.  Every step's forward vector is kept (no recompute
+ * schedule), so checkpoint_interval must be 0 or 1; the workspace holds 32 KiB
+ * per step per 32 sequences in flight (two such areas for the backward call).
  */
 bcjr_status bcjr_dense_forward(const float* w, const float* codebook, const float* log_trans,
                                float T, int n_states, int seq_len, int n_seq, float* w_hat,

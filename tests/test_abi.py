@@ -127,4 +127,7 @@ def test_dense_arguments_are_rejected_on_the_host(lib):
     assert call(opt=ctypes.pointer(o)) == UNSUPPORTED
     o.checkpoint_interval = -1
     assert call(opt=ctypes.pointer(o)) == INVALID
+    o.checkpoint_interval = 0
+    o.sequences_in_flight = 1                 # only the automatic choice (0) is accepted
+    assert call(opt=ctypes.pointer(o)) == INVALID
     assert call(N=0) == 0                     # nothing to do
