@@ -444,15 +444,32 @@ int oracle_dense_forward(const float* w, const float* c, const float* lam, doubl
 
 /* Dense VJP: the same psi/F/B formulas with pred(r) = succ(p) = all states and
  * pi(p|r) = exp(alpha_{u-1}(p) + Lam[p][r] - LSE_p'[alpha_{u-1}(p') + Lam[p'][r]]),
- * rho(s|r) = exp(Lam[r][s] + phi_{u+1}(s) + beta_{u+1}(s) - beta_u(r)). */
+ * rho(s|r) = exp(Lam[r][s] + phi_{u+1}(s) + beta_{u+1}(s) - beta_u(r)).
+ *
+ * grad_lam (optional, [S][S]): the gradient with respect to the log-transitions
+ * ("key technical innovations": exact gradients with respect to the trellis
+ * parameters).  Lam[p][r] enters the path log-weight once per transition
+ * p -> r, so dL/dLam[p][r] = Cov(G, #transitions p -> r) with
+ * G = sum_u g_u c(s_u), i.e. summed over the transitions u-1 -> u,
+ *   xi_u(p,r) = P(s_{u-1} = p, s_u = r)
+ *             = exp(alpha_{u-1}(p) + Lam[p][r] + phi_u(r) + beta_u(r) - log Z),
+ *   dL/dLam[p][r] = sum_u xi_u(p,r) (F_{u-1}(p) + e_{u-1}(p) + e_u(r) + B_u(r)),
+ * where e_u(r) = g_u (c(r) - w_hat_u) and F, B are the conditional expectations
+ * of the past and future parts of G - E[G] defined above (the Markov property
+ * splits E[G - E[G] | s_{u-1} = p, s_u = r] into those two parts). */
 int oracle_dense_backward(const float* g, const float* w, const float* c, const float* lam,
                           double T, int S, int n, int N, double* grad_w, double* grad_c,
-                          int nthreads) {
+                          double* grad_lam, int nthreads) {
   if (!dense_args_ok(S, n, N, T) || !g || !w || !c || !lam || !grad_w || !grad_c)
     return ORACLE_BAD_ARG;
   int status = ORACLE_OK;
   double* gc_seq = (double*)calloc((size_t)(N > 0 ? N : 1) * S, sizeof(double));
-  if (!gc_seq) return ORACLE_NO_MEMORY;
+  double* gl_seq = grad_lam ? (double*)calloc((size_t)(N > 0 ? N : 1) * S * S, sizeof(double)) : NULL;
+  if (!gc_seq || (grad_lam && !gl_seq)) {
+    free(gc_seq);
+    free(gl_seq);
+    return ORACLE_NO_MEMORY;
+  }
 #ifdef _OPENMP
   if (nthreads <= 0) nthreads = omp_get_max_threads();
 #pragma omp parallel for schedule(dynamic, 1) num_threads(nthreads)
@@ -461,6 +478,7 @@ int oracle_dense_backward(const float* g, const float* w, const float* c, const 
     const float* wq = w + (size_t)q * n;
     const float* gq = g + (size_t)q * n;
     double* gcq = gc_seq + (size_t)q * S;
+    double* glq = gl_seq ? gl_seq + (size_t)q * S * S : NULL;
     double* alpha = (double*)malloc(sizeof(double) * (size_t)n * S);
     double* F = (double*)malloc(sizeof(double) * (size_t)n * S);
     double* beta_t = (double*)malloc(sizeof(double) * S);
@@ -521,6 +539,18 @@ int oracle_dense_backward(const float* g, const float* w, const float* c, const 
           B_t[r] = acc;
         }
       }
+      if (glq && u >= 1) { /* transitions u-1 -> u */
+        for (int p = 0; p < S; ++p) {
+          const double ap = alpha[(size_t)(u - 1) * S + p];
+          const double past = F[(size_t)(u - 1) * S + p] + (double)gq[u - 1] * ((double)c[p] - what[u - 1]);
+          for (int r = 0; r < S; ++r) {
+            const double xi =
+                exp(ap + (double)lam[(size_t)p * S + r] + emission(wq[u], c[r], T) + beta_t[r] - lz);
+            const double future = (double)gq[u] * ((double)c[r] - what[u]) + B_t[r];
+            glq[(size_t)p * S + r] += xi * (past + future);
+          }
+        }
+      }
       double gw = 0.0;
       for (int r = 0; r < S; ++r) {
         const double gm = exp(alpha[(size_t)u * S + r] + beta_t[r] - lz);
@@ -537,7 +567,13 @@ int oracle_dense_backward(const float* g, const float* w, const float* c, const 
   for (int s = 0; s < S; ++s) grad_c[s] = 0.0;
   for (int q = 0; q < N; ++q)
     for (int s = 0; s < S; ++s) grad_c[s] += gc_seq[(size_t)q * S + s];
+  if (grad_lam) {
+    for (size_t i = 0; i < (size_t)S * S; ++i) grad_lam[i] = 0.0;
+    for (int q = 0; q < N; ++q)
+      for (size_t i = 0; i < (size_t)S * S; ++i) grad_lam[i] += gl_seq[(size_t)q * S * S + i];
+  }
   free(gc_seq);
+  free(gl_seq);
   return status;
 }
 

@@ -15,6 +15,7 @@ log-weight), with no forward or backward recursion anywhere:
 
   dL/dw_u  = (2/T) Cov(G, c(s_u))
   dL/dc(r) = sum_u g_u P(s_u = r) + (2/T) sum_u (w_u - c(r)) Cov(G, 1[s_u = r])
+  dL/dLam[p][r] = Cov(G, number of transitions p -> r on the path)      (dense)
 
 where G = sum_t g_t c(s_t).  Also the minimum-distortion (T -> 0) path.
 Sizes: S * 2^(k (n-1)) bitshift paths, S^n dense paths; keep them below ~1e6.
@@ -73,6 +74,11 @@ def _path_stats(paths, w_row, c, T, g_row=None, log_trans=None):
         grad_c = (g_row[:, None] * gamma).sum(axis=0) + (2.0 / T) * (
             (w_row[:, None] - c[None, :]) * cov_ind).sum(axis=0)
         out.update(grad_w=grad_w, grad_c=grad_c)
+        if log_trans is not None:
+            cov_tr = np.zeros((S, S))               # Cov(G, #transitions p -> r)
+            for t in range(1, n):
+                np.add.at(cov_tr, (paths[:, t - 1], paths[:, t]), p * Gc)
+            out.update(grad_lam=cov_tr)
     return out
 
 
@@ -129,4 +135,5 @@ def dense_backward(grad_w_hat, w, codebook, log_trans, T):
     lam = _as64(log_trans)
     paths = dense_paths(c.shape[0], w.shape[1])
     res = [_path_stats(paths, w[i], c, float(T), g_row=g[i], log_trans=lam) for i in range(w.shape[0])]
-    return np.stack([r["grad_w"] for r in res]), np.sum([r["grad_c"] for r in res], axis=0)
+    return (np.stack([r["grad_w"] for r in res]), np.sum([r["grad_c"] for r in res], axis=0),
+            np.sum([r["grad_lam"] for r in res], axis=0))

@@ -136,7 +136,8 @@ def dense_forward(w, codebook, log_trans, T, want_gamma=False, nthreads=0):
     return w_hat, log_z, gamma
 
 
-def dense_backward(grad_w_hat, w, codebook, log_trans, T, nthreads=0):
+def dense_backward(grad_w_hat, w, codebook, log_trans, T, nthreads=0, want_grad_lam=False):
+    """(grad_w [N][n], grad_c [S]) and, with want_grad_lam, grad_log_trans [S][S]."""
     g = _f32(grad_w_hat)
     w = _f32(w)
     c = _f32(codebook)
@@ -145,7 +146,9 @@ def dense_backward(grad_w_hat, w, codebook, log_trans, T, nthreads=0):
     S = c.shape[0]
     grad_w = np.zeros((N, n))
     grad_c = np.zeros(S)
+    grad_lam = np.zeros((S, S)) if want_grad_lam else None
     _check(_load().oracle_dense_backward(_p(g, _F), _p(w, _F), _p(c, _F), _p(lam, _F),
                                          ctypes.c_double(float(T)), S, n, N, _p(grad_w, _D),
-                                         _p(grad_c, _D), int(nthreads)), "oracle_dense_backward")
-    return grad_w, grad_c
+                                         _p(grad_c, _D), _p(grad_lam, _D) if grad_lam is not None else None,
+                                         int(nthreads)), "oracle_dense_backward")
+    return (grad_w, grad_c, grad_lam) if want_grad_lam else (grad_w, grad_c)

@@ -16,7 +16,10 @@ computation of a 1D Ising-like chain):
     translation identity sum grad_w + sum grad_c = sum g;
   * T -> 0: soft codeword -> codeword of the least-distortion path, and the
     max-sum decode equals the enumerated least-distortion path;
-  * dense trellis: brute force, and T -> inf gives gamma_t = u P^t.
+  * dense trellis: brute force, and T -> inf gives gamma_t = u P^t; the
+    log-transition gradient against brute force and finite differences, and
+    its entries sum to zero (a common shift of Lambda changes no path's
+    probability).
 """
 import os
 
@@ -229,10 +232,47 @@ def test_dense_matches_path_enumeration():
     b = brute.dense_forward(w, c, lam, T)
     for x, y in zip(a, b):
         np.testing.assert_allclose(x, y, rtol=1e-13, atol=1e-13)
-    ga = oracle.dense_backward(g, w, c, lam, T)
+    ga = oracle.dense_backward(g, w, c, lam, T, want_grad_lam=True)
     gb = brute.dense_backward(g, w, c, lam, T)
+    assert len(ga) == len(gb) == 3
     for x, y in zip(ga, gb):
         np.testing.assert_allclose(x, y, rtol=1e-11, atol=1e-12)
+
+
+def test_dense_transition_gradient_matches_finite_differences():
+    S, n, T = 8, 6, 0.5
+    lam = I.log_transition(S, seed=31)
+    c = I.codebook(S, seed=32)
+    w = I.weights(2, n, seed=33)
+    g = I.upstream_grad(2, n, seed=34)
+    _, _, grad_lam = oracle.dense_backward(g, w, c, lam, T, want_grad_lam=True)
+    g64 = g.double().numpy()
+
+    def loss(p, r):
+        def f(val):
+            ll = lam.clone()
+            ll[p, r] = float(val)
+            return float((g64 * oracle.dense_forward(w, c, ll, T)[0]).sum())
+        return f
+
+    h = 2.0 ** -9
+    scale = max(1.0, np.abs(grad_lam).max())
+    for (p, r) in [(0, 0), (3, 5), (7, 1), (5, 5), (2, 7)]:
+        fd = _five_point(loss(p, r), float(lam[p, r]), h)
+        assert abs(fd - grad_lam[p, r]) <= 1e-7 * scale, (p, r, fd, grad_lam[p, r])
+
+
+def test_dense_transition_gradient_sums_to_zero():
+    # Adding one constant to every Lambda entry adds (n-1) times it to every
+    # path's log-weight, which leaves the path distribution unchanged.
+    S, n, T = 16, 9, 0.3
+    lam = I.log_transition(S, seed=35)
+    c = I.codebook(S, seed=36)
+    w = I.weights(3, n, seed=37)
+    g = I.upstream_grad(3, n, seed=38)
+    _, _, grad_lam = oracle.dense_backward(g, w, c, lam, T, want_grad_lam=True)
+    assert abs(grad_lam.sum()) <= 1e-12 * max(1.0, np.abs(grad_lam).sum())
+    assert np.abs(grad_lam).max() > 1e-3
 
 
 def test_dense_infinite_temperature_is_a_markov_chain():
