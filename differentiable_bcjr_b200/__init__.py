@@ -23,12 +23,12 @@ __all__ = [
     "LIB_PATH", "lib", "BCJRError", "bcjr_forward", "bcjr_backward", "viterbi_decode",
     "bcjr_dense_forward", "bcjr_dense_backward", "workspace_size", "Workspace",
     "SoftTrellisQuant", "soft_quantize", "bcjr_forward_static_scratch", "OP_FORWARD", "OP_BACKWARD", "OP_VITERBI",
-    "OP_DENSE_FORWARD", "OP_DENSE_BACKWARD", "STATUS",
+    "OP_DENSE_FORWARD", "OP_DENSE_BACKWARD", "OP_DENSE_BACKWARD_LAMBDA", "STATUS",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbcjr.so")
 
-OP_FORWARD, OP_BACKWARD, OP_VITERBI, OP_DENSE_FORWARD, OP_DENSE_BACKWARD = range(5)
+OP_FORWARD, OP_BACKWARD, OP_VITERBI, OP_DENSE_FORWARD, OP_DENSE_BACKWARD, OP_DENSE_BACKWARD_LAMBDA = range(6)
 STATUS = {0: "BCJR_OK", 1: "BCJR_ERR_INVALID_ARG", 2: "BCJR_ERR_UNSUPPORTED", 3: "BCJR_ERR_WORKSPACE",
           4: "BCJR_ERR_CUDA", 5: "BCJR_ERR_TIMEOUT", 6: "BCJR_ERR_NONFINITE"}
 
@@ -60,6 +60,8 @@ _SIGS = {
     "bcjr_dense_forward": (_I, [_P, _P, _P, _F, _I, _I, _I, _P, _P, _P, ctypes.POINTER(Options), _P, _Z, _P]),
     "bcjr_dense_backward": (_I, [_P, _P, _P, _P, _P, _F, _I, _I, _I, _P, _P, _I, ctypes.POINTER(Options), _P,
                                  _Z, _P]),
+    "bcjr_dense_backward_lambda": (_I, [_P, _P, _P, _P, _P, _F, _I, _I, _I, _P, _P, _P, _I,
+                                        ctypes.POINTER(Options), _P, _Z, _P]),
     "bcjr_get_status": (_I, [_P, _P]),
     "bcjr_status_string": (ctypes.c_char_p, [_I]),
     "bcjr_version": (_I, []),
@@ -248,7 +250,10 @@ def bcjr_dense_forward(w, codebook, log_trans, T, want_marginals=False, checkpoi
     return w_hat, marg, log_z
 
 
-def bcjr_dense_backward(grad_w_hat, w, codebook, log_trans, w_hat, T, checkpoint_interval=0, ws=None):
+def bcjr_dense_backward(grad_w_hat, w, codebook, log_trans, w_hat, T, checkpoint_interval=0, ws=None,
+                        want_grad_log_trans=False):
+    """VJP of the dense soft codeword: (grad_w [N][n], grad_codebook [S]) and,
+    with want_grad_log_trans, grad_log_trans [S][S] as a third result."""
     _need_cuda(grad_w_hat, w, codebook, log_trans, w_hat)
     N, n = w.shape
     S = codebook.shape[0]
@@ -256,14 +261,22 @@ def bcjr_dense_backward(grad_w_hat, w, codebook, log_trans, w_hat, T, checkpoint
     grad_w = torch.empty((N, n), dtype=torch.float32, device=dev)
     grad_c = torch.empty((S,), dtype=torch.float32, device=dev)
     o = _opts(checkpoint_interval)
-    nbytes = lib().bcjr_workspace_size(OP_DENSE_BACKWARD, _log2_states(S), 0, n, N, ctypes.byref(o))
+    op = OP_DENSE_BACKWARD_LAMBDA if want_grad_log_trans else OP_DENSE_BACKWARD
+    nbytes = lib().bcjr_workspace_size(op, _log2_states(S), 0, n, N, ctypes.byref(o))
     if nbytes == 0:
         raise BCJRError(2, "bcjr_workspace_size")
     wsb = _ws(dev, nbytes, ws)
-    _check(lib().bcjr_dense_backward(_ptr(grad_w_hat), _ptr(w), _ptr(codebook), _ptr(log_trans), _ptr(w_hat),
-                                     float(T), S, n, N, _ptr(grad_w), _ptr(grad_c), 0, ctypes.byref(o), _ptr(wsb),
-                                     wsb.numel(), _stream(dev)), "bcjr_dense_backward")
-    return grad_w, grad_c
+    if not want_grad_log_trans:
+        _check(lib().bcjr_dense_backward(_ptr(grad_w_hat), _ptr(w), _ptr(codebook), _ptr(log_trans), _ptr(w_hat),
+                                         float(T), S, n, N, _ptr(grad_w), _ptr(grad_c), 0, ctypes.byref(o),
+                                         _ptr(wsb), wsb.numel(), _stream(dev)), "bcjr_dense_backward")
+        return grad_w, grad_c
+    grad_lam = torch.empty((S, S), dtype=torch.float32, device=dev)
+    _check(lib().bcjr_dense_backward_lambda(_ptr(grad_w_hat), _ptr(w), _ptr(codebook), _ptr(log_trans),
+                                            _ptr(w_hat), float(T), S, n, N, _ptr(grad_w), _ptr(grad_c),
+                                            _ptr(grad_lam), 0, ctypes.byref(o), _ptr(wsb), wsb.numel(),
+                                            _stream(dev)), "bcjr_dense_backward_lambda")
+    return grad_w, grad_c, grad_lam
 
 
 class SoftTrellisQuant(torch.autograd.Function):

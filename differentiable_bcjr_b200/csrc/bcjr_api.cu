@@ -131,7 +131,7 @@ const char* bcjr_status_string(bcjr_status s) {
 
 size_t bcjr_workspace_size(int op, int state_bits, int k, int seq_len, int n_seq, const bcjr_options* opt) {
   if (seq_len < 1 || n_seq < 0) return 0;
-  if (op == BCJR_OP_DENSE_FORWARD || op == BCJR_OP_DENSE_BACKWARD) {
+  if (op == BCJR_OP_DENSE_FORWARD || op == BCJR_OP_DENSE_BACKWARD || op == BCJR_OP_DENSE_BACKWARD_LAMBDA) {
     if (state_bits < 1 || state_bits > 16) return 0;
     return bcjr_dense_workspace_size_impl(op, 1 << state_bits, seq_len, n_seq, opt);
   }

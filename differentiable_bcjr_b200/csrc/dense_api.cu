@@ -15,29 +15,56 @@ constexpr size_t kAlign = 256;
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
 struct DenseLayout {
-  size_t P, PT, ckx, ckf, mtab, gc, total, ck_stride, mt_stride;
+  size_t P, PT, ckx, ckf, ckv, ckw, mtab, gc, dlpart, total, ck_stride, mt_stride;
 };
 
-DenseLayout dense_layout(int grid, int n, bool adjoint) {
+// `dl_parts` > 0 adds the rows V, W of the log-transition gradient and that
+// many [S][S] partial sums.
+DenseLayout dense_layout(int grid, int n, bool adjoint, int dl_parts = 0) {
   const size_t S = bcjr::kDenseStates, M = bcjr::kDenseRows;
   DenseLayout l = {};
   l.ck_stride = static_cast<size_t>(n) * M * S;
   l.mt_stride = static_cast<size_t>(n) * M;
+  const size_t ck_bytes = static_cast<size_t>(grid) * l.ck_stride * sizeof(float);
   size_t off = kHeader;
   l.P = off;
   off = align_up(off + S * S * sizeof(float));
   l.PT = off;
   off = align_up(off + S * S * sizeof(float));
   l.ckx = off;
-  off = align_up(off + static_cast<size_t>(grid) * l.ck_stride * sizeof(float));
+  off = align_up(off + ck_bytes);
   l.ckf = off;
-  if (adjoint) off = align_up(off + static_cast<size_t>(grid) * l.ck_stride * sizeof(float));
+  if (adjoint) off = align_up(off + ck_bytes);
+  l.ckv = off;
+  if (dl_parts > 0) off = align_up(off + ck_bytes);
+  l.ckw = off;
+  if (dl_parts > 0) off = align_up(off + ck_bytes);
   l.mtab = off;
   off = align_up(off + static_cast<size_t>(grid) * l.mt_stride * sizeof(float));
   l.gc = off;
   if (adjoint) off = align_up(off + static_cast<size_t>(grid) * S * sizeof(float));
+  l.dlpart = off;
+  off = align_up(off + static_cast<size_t>(dl_parts) * S * S * sizeof(float));
   l.total = off;
   return l;
+}
+
+// Launch geometry of the backward call that also returns the log-transition
+// gradient: the rows of that gradient live in per-CTA regions, so every CTA
+// takes one block of 32 sequences per launch and longer batches run in chunks
+// of 32 x (CTAs that fit) sequences.  `parts` = partial sums of the reduction
+// (one per SM).
+bcjr_status dlam_geometry(int N, int* grid, int* chunk, int* parts) {
+  const int cap = bcjr::dense_max_grid(true);
+  if (cap < 1) return BCJR_ERR_UNSUPPORTED;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return BCJR_ERR_CUDA;
+  const int blocks = (N + bcjr::kDenseRows - 1) / bcjr::kDenseRows;
+  *grid = blocks < 1 ? 1 : (blocks < cap ? blocks : cap);
+  *chunk = cap * bcjr::kDenseRows;
+  *parts = sms;
+  return BCJR_OK;
 }
 
 bcjr_status from_cuda(cudaError_t e) {
@@ -59,16 +86,18 @@ bcjr_status check_options(const bcjr_options* opt) {
 
 bcjr_status dense_common(bool adjoint, const float* g, const float* w, const float* c, const float* lam,
                          const float* what_in, float T, int S, int n, int N, float* w_hat, float* marginals,
-                         float* log_z, float* grad_w, float* grad_c, int accumulate, const bcjr_options* opt,
-                         void* ws, size_t ws_bytes, bcjr_stream_t stream) {
+                         float* log_z, float* grad_w, float* grad_c, float* grad_lam, int accumulate,
+                         const bcjr_options* opt, void* ws, size_t ws_bytes, bcjr_stream_t stream) {
   if (S < 1 || n < 1 || N < 0 || !(T > 0.f) || !std::isfinite(T)) return BCJR_ERR_INVALID_ARG;
   bcjr_status st = check_options(opt);
   if (st != BCJR_OK) return st;
   if (S != bcjr::kDenseStates) return BCJR_ERR_UNSUPPORTED;
+  if (grad_lam && !aligned(grad_lam, 4)) return BCJR_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (N == 0) {
     if (!adjoint || accumulate) return BCJR_OK;
     if (!grad_c) return BCJR_ERR_INVALID_ARG;
+    if (grad_lam && (st = from_cuda(cudaMemsetAsync(grad_lam, 0, S * S * sizeof(float), s))) != BCJR_OK) return st;
     return from_cuda(cudaMemsetAsync(grad_c, 0, S * sizeof(float), s));
   }
   if (!w || !c || !lam || !aligned(w, 4) || !aligned(c, 4) || !aligned(lam, 4)) return BCJR_ERR_INVALID_ARG;
@@ -79,9 +108,14 @@ bcjr_status dense_common(bool adjoint, const float* g, const float* w, const flo
     if (marginals && !aligned(marginals, 16)) return BCJR_ERR_INVALID_ARG;
   }
   if (!ws || !aligned(ws, kAlign)) return BCJR_ERR_WORKSPACE;
-  int grid = 0;
-  if ((st = from_cuda(bcjr::dense_geometry(adjoint, N, &grid))) != BCJR_OK) return st;
-  const DenseLayout lay = dense_layout(grid, n, adjoint);
+  const bool dl = adjoint && grad_lam;
+  int grid = 0, chunk = N, parts = 0;
+  if (dl) {
+    if ((st = dlam_geometry(N, &grid, &chunk, &parts)) != BCJR_OK) return st;
+  } else if ((st = from_cuda(bcjr::dense_geometry(adjoint, N, &grid))) != BCJR_OK) {
+    return st;
+  }
+  const DenseLayout lay = dense_layout(grid, n, adjoint, parts);
   if (ws_bytes < lay.total) return BCJR_ERR_WORKSPACE;
   char* base = static_cast<char*>(ws);
   bcjr::DenseParams p = {};
@@ -98,6 +132,8 @@ bcjr_status dense_common(bool adjoint, const float* g, const float* w, const flo
   p.PT = reinterpret_cast<const float*>(base + lay.PT);
   p.ckx = reinterpret_cast<float*>(base + lay.ckx);
   p.ckf = reinterpret_cast<float*>(base + lay.ckf);
+  p.ckv = dl ? reinterpret_cast<float*>(base + lay.ckv) : nullptr;
+  p.ckw = dl ? reinterpret_cast<float*>(base + lay.ckw) : nullptr;
   p.mtab = reinterpret_cast<float*>(base + lay.mtab);
   p.status = reinterpret_cast<int*>(base);
   p.ck_stride = lay.ck_stride;
@@ -107,8 +143,49 @@ bcjr_status dense_common(bool adjoint, const float* g, const float* w, const flo
   p.n = n;
   p.N = N;
   if ((st = from_cuda(cudaMemsetAsync(ws, 0, sizeof(int), s))) != BCJR_OK) return st;
-  if ((st = from_cuda(bcjr::launch_dense(p, lam, adjoint, grid, s))) != BCJR_OK) return st;
-  if (adjoint) return from_cuda(bcjr::launch_gradc_reduce(p.gc_part, grid, S, grad_c, accumulate, s));
+  if (!dl) {
+    if ((st = from_cuda(bcjr::launch_dense(p, lam, adjoint, grid, s))) != BCJR_OK) return st;
+    if (adjoint) return from_cuda(bcjr::launch_gradc_reduce(p.gc_part, grid, S, grad_c, accumulate, s));
+    return BCJR_OK;
+  }
+  // Backward call with the log-transition gradient, chunk by chunk: each
+  // chunk's backward kernel writes the rows X, U, V, W of its transitions, the
+  // tensor-core kernel sums them into per-SM partials, and the reductions add
+  // the chunk's codebook and log-transition gradients to the outputs.
+  float* dlpart = reinterpret_cast<float*>(base + lay.dlpart);
+  for (int c0 = 0; c0 < N; c0 += chunk) {
+    const int Nc = (N - c0) < chunk ? (N - c0) : chunk;
+    const int acc = (accumulate || c0 > 0) ? 1 : 0;
+    const size_t off = static_cast<size_t>(c0) * n;
+    bcjr::DenseParams pc = p;
+    pc.w = w + off;
+    pc.g = g + off;
+    pc.what_in = what_in + off;
+    pc.grad_w = grad_w + off;
+    pc.N = Nc;
+    const int grid_c = (Nc + bcjr::kDenseRows - 1) / bcjr::kDenseRows;
+    if ((st = from_cuda(bcjr::launch_dense(pc, lam, true, grid_c, s, c0 == 0))) != BCJR_OK) return st;
+    if ((st = from_cuda(bcjr::launch_gradc_reduce(pc.gc_part, grid_c, S, grad_c, acc, s))) != BCJR_OK) return st;
+    if (n == 1) {  // no transitions: the gradient is zero
+      if (!acc && (st = from_cuda(cudaMemsetAsync(grad_lam, 0, S * S * sizeof(float), s))) != BCJR_OK) return st;
+      continue;
+    }
+    bcjr::DlamParams dp = {};
+    dp.X = pc.ckx;
+    dp.U = pc.ckf;
+    dp.V = pc.ckv;
+    dp.W = pc.ckw;
+    dp.part = dlpart;
+    dp.status = pc.status;
+    dp.region_stride = static_cast<long long>(lay.ck_stride);
+    dp.spr = static_cast<long long>(n - 1) * (bcjr::kDenseRows / 8);
+    dp.total_stages = static_cast<long long>(grid_c) * dp.spr;
+    int gd = 0;
+    if ((st = from_cuda(bcjr::dlam_grid(dp.total_stages, &gd))) != BCJR_OK) return st;
+    if (gd > parts) gd = parts;
+    if ((st = from_cuda(bcjr::launch_dlam(dp, gd, s))) != BCJR_OK) return st;
+    if ((st = from_cuda(bcjr::launch_dlam_reduce(dlpart, gd, pc.P, grad_lam, acc, s))) != BCJR_OK) return st;
+  }
   return BCJR_OK;
 }
 
@@ -117,8 +194,13 @@ bcjr_status dense_common(bool adjoint, const float* g, const float* w, const flo
 size_t bcjr_dense_workspace_size_impl(int op, int n_states, int seq_len, int n_seq, const bcjr_options* opt) {
   if (n_states != bcjr::kDenseStates || seq_len < 1 || n_seq < 0) return 0;
   if (check_options(opt) != BCJR_OK) return 0;
-  const bool adjoint = (op == BCJR_OP_DENSE_BACKWARD);
+  const bool adjoint = (op == BCJR_OP_DENSE_BACKWARD || op == BCJR_OP_DENSE_BACKWARD_LAMBDA);
   int grid = 0;
+  if (op == BCJR_OP_DENSE_BACKWARD_LAMBDA) {
+    int chunk = 0, parts = 0;
+    if (dlam_geometry(n_seq > 0 ? n_seq : 1, &grid, &chunk, &parts) != BCJR_OK) return 0;
+    return dense_layout(grid, seq_len, true, parts).total;
+  }
   if (bcjr::dense_geometry(adjoint, n_seq > 0 ? n_seq : 1, &grid) != cudaSuccess) return 0;
   return dense_layout(grid, seq_len, adjoint).total;
 }
@@ -130,7 +212,7 @@ bcjr_status bcjr_dense_forward(const float* w, const float* codebook, const floa
                                float* log_z, const bcjr_options* opt, void* workspace, size_t workspace_bytes,
                                bcjr_stream_t stream) {
   return dense_common(false, nullptr, w, codebook, log_trans, nullptr, T, n_states, seq_len, n_seq, w_hat,
-                      marginals, log_z, nullptr, nullptr, 0, opt, workspace, workspace_bytes, stream);
+                      marginals, log_z, nullptr, nullptr, nullptr, 0, opt, workspace, workspace_bytes, stream);
 }
 
 bcjr_status bcjr_dense_backward(const float* grad_w_hat, const float* w, const float* codebook,
@@ -139,7 +221,18 @@ bcjr_status bcjr_dense_backward(const float* grad_w_hat, const float* w, const f
                                 const bcjr_options* opt, void* workspace, size_t workspace_bytes,
                                 bcjr_stream_t stream) {
   return dense_common(true, grad_w_hat, w, codebook, log_trans, w_hat, T, n_states, seq_len, n_seq, nullptr,
-                      nullptr, nullptr, grad_w, grad_codebook, accumulate_codebook, opt, workspace,
+                      nullptr, nullptr, grad_w, grad_codebook, nullptr, accumulate_codebook, opt, workspace,
+                      workspace_bytes, stream);
+}
+
+bcjr_status bcjr_dense_backward_lambda(const float* grad_w_hat, const float* w, const float* codebook,
+                                       const float* log_trans, const float* w_hat, float T, int n_states,
+                                       int seq_len, int n_seq, float* grad_w, float* grad_codebook,
+                                       float* grad_log_trans, int accumulate, const bcjr_options* opt,
+                                       void* workspace, size_t workspace_bytes, bcjr_stream_t stream) {
+  if (!grad_log_trans) return BCJR_ERR_INVALID_ARG;
+  return dense_common(true, grad_w_hat, w, codebook, log_trans, w_hat, T, n_states, seq_len, n_seq, nullptr,
+                      nullptr, nullptr, grad_w, grad_codebook, grad_log_trans, accumulate, opt, workspace,
                       workspace_bytes, stream);
 }
 

@@ -373,15 +373,48 @@ __global__ void __launch_bounds__(dense::Cfg<ADJ>::THREADS, 1) dense_fb_kernel(c
           }
           gw = warp_sum(gw);
           if (act[i] && lane == 0) p.grad_w[static_cast<size_t>(qg[i]) * n + t] = p.two_over_T * gw;
+          if (p.ckv && t < n - 1) {
+            // Rows of the log-transition gradient for the transition t -> t+1:
+            // X = x_t / n, U = x_t (F~_t + eps_t - D) / n with n = sum_s x_t(s) (P v_{t+1})(s)
+            // = den / zinv.  They replace this step's checkpoint, already staged.
+            const float sn = act[i] ? zinv * ginv : 0.f;
+            float X8[8], U8[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              X8[j] = x[j] * sn;
+              U8[j] = x[j] * (Fv[j] + eps[j] - Dv[i]) * sn;
+            }
+            float* xr = ckx + (static_cast<size_t>(t) * kM + q) * kS;
+            float* ur = ckf + (static_cast<size_t>(t) * kM + q) * kS;
+            *reinterpret_cast<float4*>(xr + 4 * lane) = make_float4(X8[0], X8[1], X8[2], X8[3]);
+            *reinterpret_cast<float4*>(xr + 128 + 4 * lane) = make_float4(X8[4], X8[5], X8[6], X8[7]);
+            *reinterpret_cast<float4*>(ur + 4 * lane) = make_float4(U8[0], U8[1], U8[2], U8[3]);
+            *reinterpret_cast<float4*>(ur + 128 + 4 * lane) = make_float4(U8[4], U8[5], U8[6], U8[7]);
+          }
         }
         if (t >= 1) {
           const float m2 = mtab[static_cast<size_t>(t) * kM + q];
+          float V8[8], W8[8];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const float d = wt - cs[j];
             const float v = ex2f(-(d * d) * sc2 - m2) * z[j];
             A1[a_index(st_of(lane, j), q)] = v;
-            if constexpr (ADJ) A2[a_index(st_of(lane, j), q)] = v * (eps[j] + Bt[j]);
+            V8[j] = v;
+            if constexpr (ADJ) {
+              W8[j] = v * (eps[j] + Bt[j]);
+              A2[a_index(st_of(lane, j), q)] = W8[j];
+            }
+          }
+          if constexpr (ADJ) {
+            if (p.ckv) {  // rows V = v_t, W = v_t (eps_t + B~_t) of the transition t-1 -> t
+              float* vr = p.ckv + static_cast<size_t>(blockIdx.x) * p.ck_stride + (static_cast<size_t>(t - 1) * kM + q) * kS;
+              float* wr = p.ckw + static_cast<size_t>(blockIdx.x) * p.ck_stride + (static_cast<size_t>(t - 1) * kM + q) * kS;
+              *reinterpret_cast<float4*>(vr + 4 * lane) = make_float4(V8[0], V8[1], V8[2], V8[3]);
+              *reinterpret_cast<float4*>(vr + 128 + 4 * lane) = make_float4(V8[4], V8[5], V8[6], V8[7]);
+              *reinterpret_cast<float4*>(wr + 4 * lane) = make_float4(W8[0], W8[1], W8[2], W8[3]);
+              *reinterpret_cast<float4*>(wr + 128 + 4 * lane) = make_float4(W8[4], W8[5], W8[6], W8[7]);
+            }
           }
         }
       }
@@ -431,11 +464,29 @@ cudaError_t dense_geometry(bool adjoint, int n_seq, int* grid) {
   return cudaSuccess;
 }
 
-cudaError_t launch_dense(const DenseParams& p, const float* lam, bool adjoint, int grid, cudaStream_t s) {
+int dense_max_grid(bool adjoint) {
+  const void* fn = adjoint ? reinterpret_cast<const void*>(&dense_fb_kernel<true>)
+                           : reinterpret_cast<const void*>(&dense_fb_kernel<false>);
+  const size_t smem = dense_smem_bytes(adjoint);
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+    return 0;
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  const int threads = adjoint ? dense::Cfg<true>::THREADS : dense::Cfg<false>::THREADS;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem) != cudaSuccess) return 0;
+  return per_sm * sms;
+}
+
+cudaError_t launch_dense_prep(const float* lam, const DenseParams& p, cudaStream_t s) {
   const int S = dense::kS;
   dense_prep_kernel<<<(S * S + 255) / 256, 256, 0, s>>>(lam, const_cast<float*>(p.P), const_cast<float*>(p.PT), S);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dense(const DenseParams& p, const float* lam, bool adjoint, int grid, cudaStream_t s, bool prep) {
+  cudaError_t e = cudaSuccess;
+  if (prep && (e = launch_dense_prep(lam, p, s)) != cudaSuccess) return e;
   const size_t smem = dense_smem_bytes(adjoint);
   if (adjoint) {
     dense_fb_kernel<true><<<grid, dense::Cfg<true>::THREADS, smem, s>>>(p);

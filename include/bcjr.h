@@ -71,7 +71,8 @@ typedef enum {
   BCJR_OP_BACKWARD = 1,
   BCJR_OP_VITERBI = 2,
   BCJR_OP_DENSE_FORWARD = 3,
-  BCJR_OP_DENSE_BACKWARD = 4
+  BCJR_OP_DENSE_BACKWARD = 4,
+  BCJR_OP_DENSE_BACKWARD_LAMBDA = 5
 } bcjr_op;
 
 /* Workspace bytes that a call of `op` with these sizes needs on the current
@@ -168,6 +169,27 @@ bcjr_status bcjr_dense_backward(const float* grad_w_hat, const float* w, const f
                                 int seq_len, int n_seq, float* grad_w, float* grad_codebook,
                                 int accumulate_codebook, const bcjr_options* opt, void* workspace,
                                 size_t workspace_bytes, bcjr_stream_t stream);
+
+/*
+ * bcjr_dense_backward plus the gradient with respect to the log-transitions
+ * ("key technical innovations": exact gradients with respect to the trellis
+ * parameters).  Lambda[p][r] enters the path log-weight once per transition
+ * p -> r, so with L = sum_t grad_w_hat_t w_hat_t and G = sum_t grad_w_hat_t c(s_t),
+ *   grad_log_trans[p][r] = dL/dLambda[p][r] = Cov(G, number of transitions p -> r),
+ * summed over all sequences.  grad_log_trans [n_states][n_states] is required
+ * (row = source state); with accumulate != 0 both grad_codebook and
+ * grad_log_trans are added to, otherwise overwritten.  The sum over
+ * (sequence, transition) rows runs on the tensor cores in three-pass tf32
+ * (float32-level accuracy).  Workspace: bcjr_workspace_size(BCJR_OP_DENSE_BACKWARD_LAMBDA, ...),
+ * which adds two more 32 KiB rows per step per 32 sequences in flight and a
+ * 256 KiB partial sum per SM; batches longer than 32 sequences per resident
+ * CTA run in several launches inside the call.
+ */
+bcjr_status bcjr_dense_backward_lambda(const float* grad_w_hat, const float* w, const float* codebook,
+                                       const float* log_trans, const float* w_hat, float T, int n_states,
+                                       int seq_len, int n_seq, float* grad_w, float* grad_codebook,
+                                       float* grad_log_trans, int accumulate, const bcjr_options* opt,
+                                       void* workspace, size_t workspace_bytes, bcjr_stream_t stream);
 
 /* Synchronise `stream` and return the device-side status of the most recent
  * call that used `workspace` (BCJR_OK, BCJR_ERR_NONFINITE or BCJR_ERR_TIMEOUT). */

@@ -1,0 +1,106 @@
+"""GPU parity of the log-transition gradient of the dense trellis (needs a B200).
+
+bcjr_dense_backward_lambda returns dL/dLambda next to the usual VJP; the sum
+over (sequence, transition) rows runs on the tcgen05 tensor cores in
+three-pass tf32.  Checked against the float64 oracle (itself pinned to path
+enumeration and finite differences) at lengths 1 (no transitions: zero), 2, 7
+and 64, batches that fill one CTA, leave a ragged tail and span several CTAs;
+against the zero-sum invariant (a common shift of Lambda changes no path's
+probability); and, for a batch longer than one launch, against the sum of the
+two halves computed separately.
+"""
+import numpy as np
+import pytest
+import torch
+
+import bcjr_inputs as I
+import oracle
+from parity import GRAD_REL_L2, assert_rel_l2, to_np
+
+pytestmark = pytest.mark.gpu
+
+S = 256
+
+
+@pytest.fixture(scope="module")
+def B():
+    import differentiable_bcjr_b200 as B
+    B.lib()
+    return B
+
+
+def _case(n, N, seed):
+    return (I.codebook(S, seed=500 + seed), I.weights(N, n, seed=600 + seed), I.upstream_grad(N, n, seed=700 + seed),
+            I.log_transition(S, seed=800 + seed))
+
+
+@pytest.mark.parametrize("n,N,T", [(1, 3, 0.5), (2, 5, 0.7), (7, 40, 0.2), (64, 40, 1.0), (64, 70, 0.2)])
+def test_log_transition_gradient_parity(B, n, N, T):
+    c, w, g, lam = _case(n, N, seed=n + N)
+    dc, dw, dg, dl = c.cuda(), w.cuda(), g.cuda(), lam.cuda()
+    w_hat, _, _ = B.bcjr_dense_forward(dw, dc, dl, T)
+    gw, gc, gl = B.bcjr_dense_backward(dg, dw, dc, dl, w_hat, T, want_grad_log_trans=True)
+    gw0, gc0 = B.bcjr_dense_backward(dg, dw, dc, dl, w_hat, T)
+    torch.cuda.synchronize()
+    # the extra outputs change nothing in the others
+    assert torch.equal(gw, gw0)
+    assert torch.equal(gc, gc0)
+    o_gw, o_gc, o_gl = oracle.dense_backward(g, w, c, lam, T, want_grad_lam=True)
+    if n == 1:
+        assert bool((gl == 0).all())
+        return
+    err = float(np.linalg.norm(to_np(gl) - o_gl) / np.linalg.norm(o_gl))
+    print(f"grad_log_trans rel L2 {err:.3e}")
+    assert_rel_l2(gl, o_gl, GRAD_REL_L2, "grad_log_trans")
+    # float32-level accuracy is the design (three-pass tf32); one-pass tf32
+    # would sit near 5e-4, so hold the result well below that
+    assert err < 2e-5, err
+    assert_rel_l2(gw, o_gw, GRAD_REL_L2, "grad_w")
+
+
+def test_log_transition_gradient_sums_to_zero_and_repeats(B):
+    n, N, T = 33, 300, 0.25
+    c, w, g, lam = _case(n, N, seed=3)
+    dc, dw, dg, dl = c.cuda(), w.cuda(), g.cuda(), lam.cuda()
+    w_hat, _, _ = B.bcjr_dense_forward(dw, dc, dl, T)
+    _, _, a = B.bcjr_dense_backward(dg, dw, dc, dl, w_hat, T, want_grad_log_trans=True)
+    _, _, b = B.bcjr_dense_backward(dg, dw, dc, dl, w_hat, T, want_grad_log_trans=True)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)  # fixed-order reduction: run-to-run identical
+    x = a.double()
+    assert abs(float(x.sum())) <= 1e-5 * float(x.abs().sum())
+    assert float(x.abs().max()) > 0
+
+
+def test_log_transition_gradient_over_several_launches(B):
+    # More sequences than one launch holds (32 per resident CTA): the call runs
+    # in chunks and accumulates; compare with the two halves computed apart.
+    B.lib()
+    n, T = 3, 0.4
+    import ctypes
+    o = B._opts(0)
+    # find the chunk length: the smallest N whose workspace stops growing with N
+    chunk = None
+    prev = B.lib().bcjr_workspace_size(B.OP_DENSE_BACKWARD_LAMBDA, 8, 0, n, 32, ctypes.byref(o))
+    for N in range(64, 32 * 1024 + 1, 32):
+        cur = B.lib().bcjr_workspace_size(B.OP_DENSE_BACKWARD_LAMBDA, 8, 0, n, N, ctypes.byref(o))
+        if cur == prev:
+            chunk = N - 32
+            break
+        prev = cur
+    assert chunk is not None and chunk % 32 == 0
+    N = chunk + 40
+    c, w, g, lam = _case(n, N, seed=4)
+    dc, dw, dg, dl = c.cuda(), w.cuda(), g.cuda(), lam.cuda()
+    w_hat, _, _ = B.bcjr_dense_forward(dw, dc, dl, T)
+    gw, gc, gl = B.bcjr_dense_backward(dg, dw, dc, dl, w_hat, T, want_grad_log_trans=True)
+    parts = []
+    for sl in (slice(0, chunk), slice(chunk, N)):
+        parts.append(B.bcjr_dense_backward(dg[sl].contiguous(), dw[sl].contiguous(), dc, dl,
+                                           w_hat[sl].contiguous(), T, want_grad_log_trans=True))
+    torch.cuda.synchronize()
+    assert torch.equal(gw, torch.cat([parts[0][0], parts[1][0]]))
+    ref_c = (parts[0][1].double() + parts[1][1].double())
+    ref_l = (parts[0][2].double() + parts[1][2].double())
+    assert float((gc.double() - ref_c).norm() / ref_c.norm()) < 1e-6
+    assert float((gl.double() - ref_l).norm() / ref_l.norm()) < 1e-6
