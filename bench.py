@@ -62,6 +62,8 @@ def parse():
     ap.add_argument("--workload", default="projection", choices=["projection", "dense", "viterbi"],
                     help="projection: the S=2^16, k=2 headline; dense: the 256-state fully connected trellis; "
                          "viterbi: hard decode of the projection")
+    ap.add_argument("--with-lambda", action="store_true",
+                    help="dense workload: the backward call also returns dL/dLambda (tensor-core reduction)")
     return ap.parse_args()
 
 
@@ -433,12 +435,20 @@ def run_dense(args):
     ws_f, ws_b = B.Workspace(dev), B.Workspace(dev)
     stream = torch.cuda.current_stream(dev)
 
+    wl = bool(args.with_lambda)
+
+    def backward(g_in, w_in, w_hat):
+        r = B.bcjr_dense_backward(g_in, w_in, c, lam, w_hat, T, ws=ws_b, want_grad_log_trans=wl)
+        if world > 1:
+            torch.distributed.all_reduce(r[1])
+            if wl:
+                torch.distributed.all_reduce(r[2])
+        return r
+
     def step(w_in, g_in):
         w_hat, _, _ = B.bcjr_dense_forward(w_in, c, lam, T, ws=ws_f)
-        gw, gc = B.bcjr_dense_backward(g_in, w_in, c, lam, w_hat, T, ws=ws_b)
-        if world > 1:
-            torch.distributed.all_reduce(gc)
-        return w_hat, gw, gc
+        r = backward(g_in, w_in, w_hat)
+        return w_hat, r[0], r[1]
 
     def barrier():
         if world > 1:
@@ -456,12 +466,23 @@ def run_dense(args):
         ev[i][0].record(stream)
         w_hat, _, _ = B.bcjr_dense_forward(w, c, lam, T, ws=ws_f)
         ev[i][1].record(stream)
-        gw, gc = B.bcjr_dense_backward(g, w, c, lam, w_hat, T, ws=ws_b)
+        r = B.bcjr_dense_backward(g, w, c, lam, w_hat, T, ws=ws_b, want_grad_log_trans=wl)
         ev[i][2].record(stream)
         if world > 1:
-            torch.distributed.all_reduce(gc)
+            torch.distributed.all_reduce(r[1])
+            if wl:
+                torch.distributed.all_reduce(r[2])
     barrier()
     clocks = sampler.stop()
+    plain_bwd_ms = None
+    if wl:  # the same backward call without dL/dLambda, for the cost of the extra output (not in `value`)
+        pe = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        pe[0].record(stream)
+        for _ in range(args.steps):
+            B.bcjr_dense_backward(g, w, c, lam, w_hat, T, ws=ws_b)
+        pe[1].record(stream)
+        barrier()
+        plain_bwd_ms = pe[0].elapsed_time(pe[1]) / args.steps
     fwd_ms = [a.elapsed_time(b) for a, b, _ in ev]
     bwd_ms = [b.elapsed_time(cc) for _, b, cc in ev]
     elapsed_ms = ev[0][0].elapsed_time(ev[-1][2])
@@ -507,22 +528,37 @@ def run_dense(args):
         fp32_peak = 2 * FP32_FMA_PER_CLK_PER_SM * sms * max_mhz * 1e6     # FLOP/s
         bwd_s = statistics.mean(bwd_ms) / 1e3
         fwd_s = statistics.mean(fwd_ms) / 1e3
+        # the SIMT roofline is the adjoint kernel's: without the dL/dLambda extras
+        adj_s = plain_bwd_ms / 1e3 if wl else bwd_s
         flops_b = 2 * 4 * N * n * S * S   # adjoint: two stacked contractions per sweep, two sweeps
         flops_f = 2 * 2 * N * n * S * S   # forward call: one contraction per sweep, two sweeps
         line = {
             "metric": DENSE_METRIC, "value": value, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": _dense_config(world, N),
-            "roofline": {"bound": "alu", "pipe": "FP32 FMA (SIMT)", "achieved": flops_b / bwd_s / 1e12,
-                         "peak": fp32_peak / 1e12, "unit": "TFLOP/s", "frac": flops_b / bwd_s / fp32_peak,
+            "roofline": {"bound": "alu", "pipe": "FP32 FMA (SIMT)", "achieved": flops_b / adj_s / 1e12,
+                         "peak": fp32_peak / 1e12, "unit": "TFLOP/s", "frac": flops_b / adj_s / fp32_peak,
                          "traffic": None, "kernel": "dense_fb_kernel<adjoint> (bcjr_dense_backward)",
                          "peak_source": f"2 x {FP32_FMA_PER_CLK_PER_SM} FMA/clk/SM x {sms} SMs x {max_mhz:.0f} MHz"},
             "forward_call": {"ms": 1e3 * fwd_s, "TFLOP/s": flops_f / fwd_s / 1e12,
                              "frac": flops_f / fwd_s / fp32_peak},
-            "kernels_ms": {"bcjr_dense_forward": 1e3 * fwd_s, "bcjr_dense_backward": 1e3 * bwd_s},
-            "gpu_launches": 5 * args.steps,
+            "kernels_ms": {"bcjr_dense_forward": 1e3 * fwd_s,
+                           ("bcjr_dense_backward_lambda" if wl else "bcjr_dense_backward"): 1e3 * bwd_s},
+            "gpu_launches": (8 if wl else 5) * args.steps,
             "clocks": clocks,
         }
+        if wl:
+            # dL/dLambda: sum over N (n-1) rows of P (.) (X^T W + U^T V), run as three
+            # tf32 products per operand pair on the tensor cores.
+            rows = N * (n - 1)
+            line["metric"] = DENSE_METRIC.replace("fwd+bwd", "fwd+bwd+dLambda")
+            line["config"]["lambda_gradient"] = True
+            line["lambda_gradient"] = {
+                "plain_backward_ms": plain_bwd_ms, "extra_ms": 1e3 * bwd_s - plain_bwd_ms,
+                "tensor_TFLOP_per_s_lower_bound": 3 * 2 * 2 * rows * S * S / (bwd_s - adj_s) / 1e12,
+                "algorithmic_TFLOP": 2 * 2 * rows * S * S / 1e12,
+                "tensor_TFLOP_3xtf32": 3 * 2 * 2 * rows * S * S / 1e12,
+                "kernel": "dense_dlam_kernel (tcgen05.mma kind::tf32, accumulator in TMEM)"}
         if e2e is not None:
             line["e2e"] = e2e
         if world == 1 and not args.no_cpu_baseline:
