@@ -10,7 +10,8 @@ the calls raise.
   bcjr_backward(grad_w_hat, w, codebook, w_hat, T, state_bits, k) -> (grad_w, grad_codebook)
   viterbi_decode(w, codebook, state_bits, k)          -> (states, w_hard)
   bcjr_dense_forward / bcjr_dense_backward            (fully connected trellis)
-  SoftTrellisQuant                                    torch.autograd.Function
+  bcjr_dense_backward(..., want_grad_log_trans=True)  (also dL/dLambda, tensor cores)
+  SoftTrellisQuant, DenseTrellisQuant                 torch.autograd.Function
 """
 from __future__ import annotations
 
@@ -22,7 +23,8 @@ import torch
 __all__ = [
     "LIB_PATH", "lib", "BCJRError", "bcjr_forward", "bcjr_backward", "viterbi_decode",
     "bcjr_dense_forward", "bcjr_dense_backward", "workspace_size", "Workspace",
-    "SoftTrellisQuant", "soft_quantize", "bcjr_forward_static_scratch", "OP_FORWARD", "OP_BACKWARD", "OP_VITERBI",
+    "SoftTrellisQuant", "soft_quantize", "DenseTrellisQuant", "dense_soft_quantize", "bcjr_forward_static_scratch",
+    "OP_FORWARD", "OP_BACKWARD", "OP_VITERBI",
     "OP_DENSE_FORWARD", "OP_DENSE_BACKWARD", "OP_DENSE_BACKWARD_LAMBDA", "STATUS",
 ]
 
@@ -301,3 +303,31 @@ class SoftTrellisQuant(torch.autograd.Function):
 
 def soft_quantize(w, codebook, T, state_bits, k):
     return SoftTrellisQuant.apply(w, codebook, T, state_bits, k)
+
+
+class DenseTrellisQuant(torch.autograd.Function):
+    """w_hat = soft codeword of w over the dense 256-state trellis with
+    log-transitions `log_trans` (differentiable in w, codebook and log_trans;
+    the log_trans gradient is computed only when it is required)."""
+
+    @staticmethod
+    def forward(ctx, w, codebook, log_trans, T):
+        w_c, c_c, l_c = w.contiguous(), codebook.contiguous(), log_trans.contiguous()
+        w_hat, _, _ = bcjr_dense_forward(w_c, c_c, l_c, T)
+        ctx.save_for_backward(w_c, c_c, l_c, w_hat)
+        ctx.T = float(T)
+        return w_hat
+
+    @staticmethod
+    def backward(ctx, grad_w_hat):
+        w, c, lam, w_hat = ctx.saved_tensors
+        g = grad_w_hat.contiguous().float()
+        if ctx.needs_input_grad[2]:
+            gw, gc, gl = bcjr_dense_backward(g, w, c, lam, w_hat, ctx.T, want_grad_log_trans=True)
+        else:
+            (gw, gc), gl = bcjr_dense_backward(g, w, c, lam, w_hat, ctx.T), None
+        return gw, gc, gl, None
+
+
+def dense_soft_quantize(w, codebook, log_trans, T):
+    return DenseTrellisQuant.apply(w, codebook, log_trans, T)

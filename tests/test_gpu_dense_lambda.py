@@ -104,3 +104,22 @@ def test_log_transition_gradient_over_several_launches(B):
     ref_l = (parts[0][2].double() + parts[1][2].double())
     assert float((gc.double() - ref_c).norm() / ref_c.norm()) < 1e-6
     assert float((gl.double() - ref_l).norm() / ref_l.norm()) < 1e-6
+
+
+def test_dense_autograd_function(B):
+    n, N, T = 12, 35, 0.3
+    c, w, g, lam = _case(n, N, seed=5)
+    wv = w.cuda().requires_grad_(True)
+    cv = c.cuda().requires_grad_(True)
+    lv = lam.cuda().requires_grad_(True)
+    w_hat = B.dense_soft_quantize(wv, cv, lv, T)
+    (w_hat * g.cuda()).sum().backward()
+    o_gw, o_gc, o_gl = oracle.dense_backward(g, w, c, lam, T, want_grad_lam=True)
+    assert_rel_l2(wv.grad, o_gw, GRAD_REL_L2, "grad_w")
+    assert_rel_l2(cv.grad, o_gc, GRAD_REL_L2, "grad_c")
+    assert_rel_l2(lv.grad, o_gl, GRAD_REL_L2, "grad_log_trans")
+    # without a log_trans gradient the plain backward call runs
+    lv2 = lam.cuda()
+    w2 = w.cuda().requires_grad_(True)
+    (B.dense_soft_quantize(w2, c.cuda(), lv2, T) * g.cuda()).sum().backward()
+    assert torch.equal(w2.grad, wv.grad)
