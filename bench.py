@@ -204,28 +204,40 @@ def load_peaks():
         return {}
 
 
-def kernel_source_hash():
-    """Hash of the sources that define the forward-backward kernels."""
+# Sources that define each measured kernel (its ncu counters go stale when they change).
+FB_SOURCES = ("fb_", "bcjr_device", "team", "bcjr_internal")
+VITERBI_SOURCES = ("viterbi_kernel", "bitshift_kernels", "bcjr_device", "team", "bcjr_internal")
+DENSE_SOURCES = ("dense_kernel", "bcjr_device", "bcjr_internal")
+
+
+def kernel_source_hash(prefixes=FB_SOURCES):
+    """Hash of the kernel sources whose file names start with `prefixes`."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "differentiable_bcjr_b200", "csrc")
     for f in sorted(os.listdir(d)):
-        if f.startswith(("fb_", "bcjr_device", "team", "bcjr_internal")):
+        if f.startswith(prefixes):
             h.update(f.encode())
             h.update(open(os.path.join(d, f), "rb").read())
     return h.hexdigest()[:16]
 
 
-def load_traffic():
-    """DRAM bytes per launch from the committed ncu summary, or {} once the kernels changed."""
-    p = os.path.join(ROOT, "profiles", "fb_kernel_L16_k2_full.md")
+def load_traffic(profile="fb_kernel_L16_k2_full.md", prefixes=FB_SOURCES):
+    """DRAM bytes per launch from a committed ncu summary, or {} once the kernel changed."""
+    p = os.path.join(ROOT, "profiles", profile)
     try:
         text = open(p).read()
     except OSError:
         return {}
     m = re.search(r"^kernel_source_sha256_16: (\w+)", text, re.M)
-    if not m or m.group(1) != kernel_source_hash():
+    if not m or m.group(1) != kernel_source_hash(prefixes):
         return {}
     return {k: int(v) for k, v in re.findall(r"^(\w+_dram_bytes_per_launch): (\d+)", text, re.M)}
+
+
+def scaled_traffic(bytes_full, n_seq, n_seq_full):
+    """A summary's bytes for the full launch, scaled to a launch of n_seq
+    sequences (traffic is per sequence); None when the summary is stale."""
+    return None if bytes_full is None else int(bytes_full * n_seq / n_seq_full)
 
 
 def run_gpu(args):
@@ -352,7 +364,7 @@ def run_gpu(args):
         bwd_avg_s = statistics.mean(bwd_ms) / 1e3
         fwd_avg_s = statistics.mean(fwd_ms) / 1e3
         achieved = 2 * state_steps / bwd_avg_s
-        traffic = load_traffic().get("bwd_dram_bytes_per_launch")
+        traffic = scaled_traffic(load_traffic().get("bwd_dram_bytes_per_launch"), N, I.WORKLOADS[WORKLOAD]["n_seq"])
         frac_total = ALG_MUFU_PER_STATE_STEP * state_steps * world / (ms_per_step / 1e3) / (mufu_peak * world)
         line = {
             "metric": METRIC, "value": value, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
@@ -538,7 +550,9 @@ def run_dense(args):
             "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": _dense_config(world, N),
             "roofline": {"bound": "alu", "pipe": "FP32 FMA (SIMT)", "achieved": flops_b / adj_s / 1e12,
                          "peak": fp32_peak / 1e12, "unit": "TFLOP/s", "frac": flops_b / adj_s / fp32_peak,
-                         "traffic": None, "kernel": "dense_fb_kernel<adjoint> (bcjr_dense_backward)",
+                         "traffic": scaled_traffic(load_traffic("dense_fb_kernel_S256_full.md", DENSE_SOURCES).get(
+                             "adjoint_dram_bytes_per_launch"), N, W["n_seq"]),
+                         "kernel": "dense_fb_kernel<adjoint> (bcjr_dense_backward)",
                          "peak_source": f"2 x {FP32_FMA_PER_CLK_PER_SM} FMA/clk/SM x {sms} SMs x {max_mhz:.0f} MHz"},
             "forward_call": {"ms": 1e3 * fwd_s, "TFLOP/s": flops_f / fwd_s / 1e12,
                              "frac": flops_f / fwd_s / fp32_peak},
@@ -661,7 +675,10 @@ def run_viterbi(args):
             "config": dict(_config(world, 1, N), workload=f"{WORKLOAD} (hard decode)"),
             "roofline": {"bound": "alu", "pipe": "FP64", "achieved": ops / (ms_per_step / 1e3) / 1e12,
                          "peak": fp64_peak / 1e12, "unit": "T fp64 op/s",
-                         "frac": ops / (ms_per_step / 1e3) / fp64_peak, "traffic": None,
+                         "frac": ops / (ms_per_step / 1e3) / fp64_peak,
+                         "traffic": scaled_traffic(load_traffic("bench_viterbi_proj2048x8192_L16_k2.md",
+                                                                VITERBI_SOURCES).get("viterbi_dram_bytes_per_launch"),
+                                                   N, I.WORKLOADS[WORKLOAD]["n_seq"]),
                          "kernel": "viterbi_kernel (viterbi_decode)",
                          "peak_source": f"{FP64_OPS_PER_CLK_PER_SM} fp64 lanes/clk/SM x {sms} SMs x {max_mhz:.0f} MHz"},
             "kernels_ms": {"viterbi_decode": ms_per_step},
