@@ -27,7 +27,8 @@ def declared_functions():
 def test_header_declares_the_calls():
     names = declared_functions()
     for required in ["bcjr_forward", "bcjr_backward", "viterbi_decode", "bcjr_workspace_size",
-                     "bcjr_get_status", "bcjr_status_string", "bcjr_dense_forward", "bcjr_dense_backward"]:
+                     "bcjr_get_status", "bcjr_status_string", "bcjr_dense_forward", "bcjr_dense_backward",
+                     "bcjr_dense_backward_lambda", "bcjr_forward_static_scratch"]:
         assert required in names, names
 
 
@@ -131,3 +132,22 @@ def test_dense_arguments_are_rejected_on_the_host(lib):
     o.sequences_in_flight = 1                 # only the automatic choice (0) is accepted
     assert call(opt=ctypes.pointer(o)) == INVALID
     assert call(N=0) == 0                     # nothing to do
+
+
+def test_dense_lambda_arguments_are_rejected_on_the_host(lib):
+    INVALID, UNSUPPORTED = 1, 2
+    f = lib.bcjr_dense_backward_lambda
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p] * 5 + [ctypes.c_float] + [ctypes.c_int] * 3 + [ctypes.c_void_p] * 3 + \
+        [ctypes.c_int, ctypes.POINTER(_Opts), ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+
+    def call(S=256, n=4, N=2, T=0.5, g=4096, w=8192, c=12288, lam=16384, what=20480, gw=24576, gc=28672,
+             gl=32768, ws=65536):
+        return f(g, w, c, lam, what, T, S, n, N, gw, gc, gl, 0, None, ws, 1 << 20, None)
+
+    assert call(gl=0) == INVALID              # the log-transition gradient is this call's output
+    assert call(gl=32770) == INVALID          # misaligned
+    assert call(T=-1.0) == INVALID
+    assert call(S=64) == UNSUPPORTED
+    assert call(g=0) == INVALID
+    assert call(gc=0) == INVALID
