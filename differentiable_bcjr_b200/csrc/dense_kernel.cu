@@ -25,8 +25,8 @@
 // in shared memory (column-major, 16-byte slots XOR-swizzled so that both the
 // row-broadcast reads and the transposing writes are conflict-free) and P or
 // P^T streams through a double-buffered shared-memory window of 32 rows with
-// cp.async.  A thread holds RQ sequences x 8 states (states 4l..4l+3 and
-// 128+4l..128+4l+3 of lane l), so state sums are warp shuffles; the
+// cp.async.  A thread holds 4 sequences x 8 states (states 4l..4l+3 and
+// 128+4l..128+4l+3 of lane l), 8 warps per CTA, so state sums are warp shuffles; the
 // contraction runs on packed f32x2 fused multiply-adds over state pairs (each
 // lane rounds exactly as a scalar fma would).
 #include <cuda_runtime.h>
@@ -47,7 +47,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 template <bool ADJ>
 struct Cfg {
-  static constexpr int RQ = ADJ ? 4 : 8;  // sequences per thread
+  static constexpr int RQ = 4;  // sequences per thread (8 warps per CTA)
   static constexpr int WARPS = kM / RQ;
   static constexpr int THREADS = 32 * WARPS;
 };
