@@ -253,15 +253,19 @@ def bcjr_dense_forward(w, codebook, log_trans, T, want_marginals=False, checkpoi
 
 
 def bcjr_dense_backward(grad_w_hat, w, codebook, log_trans, w_hat, T, checkpoint_interval=0, ws=None,
-                        want_grad_log_trans=False):
+                        want_grad_log_trans=False, grad_codebook=None, grad_log_trans=None, accumulate=False):
     """VJP of the dense soft codeword: (grad_w [N][n], grad_codebook [S]) and,
-    with want_grad_log_trans, grad_log_trans [S][S] as a third result."""
-    _need_cuda(grad_w_hat, w, codebook, log_trans, w_hat)
+    with want_grad_log_trans, grad_log_trans [S][S] as a third result.  Given
+    `grad_codebook` / `grad_log_trans` tensors, the results go there, added to
+    their contents when `accumulate` is set."""
+    _need_cuda(grad_w_hat, w, codebook, log_trans, w_hat, grad_codebook, grad_log_trans)
     N, n = w.shape
     S = codebook.shape[0]
     dev = w.device
     grad_w = torch.empty((N, n), dtype=torch.float32, device=dev)
-    grad_c = torch.empty((S,), dtype=torch.float32, device=dev)
+    if grad_codebook is None or (want_grad_log_trans and grad_log_trans is None):
+        accumulate = False
+    grad_c = grad_codebook if grad_codebook is not None else torch.empty((S,), dtype=torch.float32, device=dev)
     o = _opts(checkpoint_interval)
     op = OP_DENSE_BACKWARD_LAMBDA if want_grad_log_trans else OP_DENSE_BACKWARD
     nbytes = lib().bcjr_workspace_size(op, _log2_states(S), 0, n, N, ctypes.byref(o))
@@ -270,14 +274,16 @@ def bcjr_dense_backward(grad_w_hat, w, codebook, log_trans, w_hat, T, checkpoint
     wsb = _ws(dev, nbytes, ws)
     if not want_grad_log_trans:
         _check(lib().bcjr_dense_backward(_ptr(grad_w_hat), _ptr(w), _ptr(codebook), _ptr(log_trans), _ptr(w_hat),
-                                         float(T), S, n, N, _ptr(grad_w), _ptr(grad_c), 0, ctypes.byref(o),
-                                         _ptr(wsb), wsb.numel(), _stream(dev)), "bcjr_dense_backward")
+                                         float(T), S, n, N, _ptr(grad_w), _ptr(grad_c), int(bool(accumulate)),
+                                         ctypes.byref(o), _ptr(wsb), wsb.numel(), _stream(dev)),
+               "bcjr_dense_backward")
         return grad_w, grad_c
-    grad_lam = torch.empty((S, S), dtype=torch.float32, device=dev)
+    grad_lam = grad_log_trans if grad_log_trans is not None else torch.empty((S, S), dtype=torch.float32,
+                                                                             device=dev)
     _check(lib().bcjr_dense_backward_lambda(_ptr(grad_w_hat), _ptr(w), _ptr(codebook), _ptr(log_trans),
                                             _ptr(w_hat), float(T), S, n, N, _ptr(grad_w), _ptr(grad_c),
-                                            _ptr(grad_lam), 0, ctypes.byref(o), _ptr(wsb), wsb.numel(),
-                                            _stream(dev)), "bcjr_dense_backward_lambda")
+                                            _ptr(grad_lam), int(bool(accumulate)), ctypes.byref(o), _ptr(wsb),
+                                            wsb.numel(), _stream(dev)), "bcjr_dense_backward_lambda")
     return grad_w, grad_c, grad_lam
 
 

@@ -34,7 +34,8 @@ def _case(n, N, seed):
             I.log_transition(S, seed=800 + seed))
 
 
-@pytest.mark.parametrize("n,N,T", [(1, 3, 0.5), (2, 5, 0.7), (7, 40, 0.2), (64, 40, 1.0), (64, 70, 0.2)])
+@pytest.mark.parametrize("n,N,T", [(1, 3, 0.5), (2, 5, 0.7), (7, 40, 0.2), (64, 40, 1.0), (64, 70, 0.2),
+                                   (16, 33, 0.02)])
 def test_log_transition_gradient_parity(B, n, N, T):
     c, w, g, lam = _case(n, N, seed=n + N)
     dc, dw, dg, dl = c.cuda(), w.cuda(), g.cuda(), lam.cuda()
@@ -143,3 +144,18 @@ def test_log_transition_gradient_full_workload(B):
     x = gl.double()
     assert bool(torch.isfinite(x).all())
     assert abs(float(x.sum())) <= 1e-5 * float(x.abs().sum())
+
+
+def test_log_transition_gradient_accumulates(B):
+    n, N, T = 9, 37, 0.35
+    c, w, g, lam = _case(n, N, seed=6)
+    dc, dw, dg, dl = c.cuda(), w.cuda(), g.cuda(), lam.cuda()
+    w_hat, _, _ = B.bcjr_dense_forward(dw, dc, dl, T)
+    _, gc1, gl1 = B.bcjr_dense_backward(dg, dw, dc, dl, w_hat, T, want_grad_log_trans=True)
+    gc = torch.full((S,), 0.25, device="cuda")
+    gl = torch.full((S, S), -0.5, device="cuda")
+    B.bcjr_dense_backward(dg, dw, dc, dl, w_hat, T, want_grad_log_trans=True, grad_codebook=gc,
+                          grad_log_trans=gl, accumulate=True)
+    torch.cuda.synchronize()
+    torch.testing.assert_close(gc, gc1 + 0.25, rtol=0, atol=1e-6)
+    torch.testing.assert_close(gl, gl1 - 0.5, rtol=0, atol=1e-6)
