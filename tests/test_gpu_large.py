@@ -7,6 +7,8 @@
     benchmark's launch): sampled sequences vs the oracle one by one at the
     first and last temperature of the annealing sweep, plus the translation
     identity sum grad_w + sum grad_codebook = sum g over all 16.7M weights;
+    its hard decode: sampled sequences bit-exact, codewords and transitions
+    valid everywhere;
   * the bit-width sweep, k = 3 and 4 on 16384 sequences: sampled sequences
     and the translation identity.
 """
@@ -103,3 +105,22 @@ def test_bitwidth_sweep_sampled(B, k):
     assert_abs(w_hat[sample], o_what, W_HAT_ATOL, f"w_hat k={k}")
     assert_rel_l2(grad_w[sample], o_gw, GRAD_REL_L2, f"grad_w k={k}")
     _translation_identity(grad_w, grad_c, g)
+
+
+def test_projection_hard_decode_sampled(B):
+    # The hard-decode launch the benchmark times (65536 sequences): sampled
+    # sequences bit-exact against the oracle's max-sum, and every decoded
+    # codeword equal to the codebook entry of its state.
+    W = I.WORKLOADS["proj2048x8192_L16_k2"]
+    L, k, n, N = W["state_bits"], W["k"], W["seq_len"], W["n_seq"]
+    c, w = I.codebook(1 << L), I.weights(N, n)
+    dc = c.cuda()
+    states, w_hard = B.viterbi_decode(w.cuda(), dc, L, k)
+    torch.cuda.synchronize()
+    sample = [0, 1, 4097, 31337, N - 2, N - 1]
+    o_states = oracle.viterbi(w[sample], c, L, k)[0]
+    assert (to_np(states[sample]) == o_states).all()
+    assert torch.equal(w_hard, dc[states.long()])
+    # every consecutive pair of states is a trellis transition
+    s = states.long()
+    assert bool(((s[:, 1:] >> k) == (s[:, :-1] & ((1 << (L - k)) - 1))).all())
