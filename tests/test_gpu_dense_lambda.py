@@ -143,7 +143,11 @@ def test_log_transition_gradient_full_workload(B):
     assert torch.equal(gl, gl2)
     x = gl.double()
     assert bool(torch.isfinite(x).all())
-    assert abs(float(x.sum())) <= 1e-5 * float(x.abs().sum())
+    # Each CTA accumulates about N (n-1) / 148 = 113k rows (6 tf32 products
+    # per row pair, float32 accumulator), so rounding leaves each entry a
+    # random-walk error near sqrt(6 * 113k) * 2^-24 ~ 5e-5 of its size.  The
+    # exact sum is zero; allow ten times that walk.
+    assert abs(float(x.sum())) <= 5e-4 * float(x.abs().sum())
 
 
 def test_log_transition_gradient_accumulates(B):
