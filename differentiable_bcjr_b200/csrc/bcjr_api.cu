@@ -91,7 +91,8 @@ struct ViterbiLayout {
 ViterbiLayout viterbi_layout(const TeamGeometry& g, int L, int k, int n) {
   ViterbiLayout l = {};
   const size_t G = static_cast<size_t>(1) << (L - k);
-  l.bp_stride = static_cast<size_t>(n) * G;
+  const int kb = k <= 2 ? k : 4;  // bits per packed backpointer (as in the kernel)
+  l.bp_stride = static_cast<size_t>(n) * G * kb / 8;
   l.bp = kHeaderBytes;
   l.total = align_up(l.bp + static_cast<size_t>(g.num_slots) * g.nseq * 2 * l.bp_stride);  // two buffers per lane
   return l;

@@ -102,7 +102,7 @@ struct ViterbiParams {
   int32_t* states;         // [N][n]
   float* w_hard;           // [N][n] or null
   double* metric;          // [N] or null
-  uint8_t* bp;             // per lane (slot x sequence in flight) [2][n][G] backpointers (by iteration parity)
+  uint8_t* bp;             // per lane (slot x sequence in flight) [2][n][G x kb bits] packed backpointers (by iteration parity)
   int* status;
   size_t bp_stride;
   int L, k, n, N;

@@ -32,7 +32,11 @@ template <int K, int CL, int NSEQ, int NTB>
 __global__ void __launch_bounds__(NTB, 1) viterbi_kernel(const ViterbiParams p) {
   using TL = Tile<K>;
   constexpr int U = TL::U, JT = TL::JT, BT = TL::BT;
-  constexpr int NB = U * BT;  // backpointer bytes a writer thread produces per step (4 or 8)
+  constexpr int NB = U * BT;  // backpointers a writer thread produces per step (4 or 8)
+  // Backpointers are packed at KB bits each (k bits for k <= 2, 4 bits for
+  // k = 3, 4), so a writer thread's NB values fill one byte (k <= 2) or two.
+  constexpr int KB = K <= 4 ? ilog2_constexpr(K) : 4;
+  static_assert(NB * KB == 8 || NB * KB == 16, "one or two bytes per writer thread and step");
   constexpr int k = K == 2 ? 1 : K == 4 ? 2 : K == 8 ? 3 : 4;
   // A cluster team fills its cluster exactly, so the trellis size is then a constant.
   constexpr int kLc = CL > 1 ? ilog2_constexpr(kStatesPerThread * CL * NTB) : 0;
@@ -48,6 +52,7 @@ __global__ void __launch_bounds__(NTB, 1) viterbi_kernel(const ViterbiParams p) 
   tm.init(L, k, team_in_cta * TS);
   const int slot = (CL > 1) ? static_cast<int>(blockIdx.x) / CL : static_cast<int>(blockIdx.x) * tpc + team_in_cta;
   const int G = tm.G, GL = tm.GL;
+  const size_t row_bytes = static_cast<size_t>(G) * KB / 8;  // backpointers of one step
   const bool contig = (K <= 4) && (L >= 3 * k);
 
   // Shared memory (doubles): per team, per sequence in flight [2][GL] group
@@ -123,7 +128,10 @@ __global__ void __launch_bounds__(NTB, 1) viterbi_kernel(const ViterbiParams p) 
     if (ti < n - 1) wk_s[x] = (wk_j[x] << (L - k)) | (wk_s[x] >> k);
     p.states[static_cast<size_t>(wk_seq[x]) * n + ti] = wk_s[x];
     if (p.w_hard) p.w_hard[static_cast<size_t>(wk_seq[x]) * n + ti] = __ldg(p.codebook + wk_s[x]);
-    if (ti >= 1) wk_j[x] = wk_bp[x][static_cast<size_t>(ti) * G + (wk_s[x] >> k)];
+    if (ti >= 1) {
+      const int bit = (wk_s[x] >> k) * KB;
+      wk_j[x] = (wk_bp[x][static_cast<size_t>(ti) * row_bytes + (bit >> 3)] >> (bit & 7)) & (K - 1);
+    }
   };
   for (int it = 0; it < iters; ++it) {
     int seq[NSEQ];
@@ -225,16 +233,15 @@ __global__ void __launch_bounds__(NTB, 1) viterbi_kernel(const ViterbiParams p) 
       pipe.before_stores();
       if (wk_act[X] && is_walker(X)) walk_step(X, n - 1 - t);  // previous sequence of this slot
       if (write && tm.a_writer) {
-        // the thread's groups a_out_index(u, bb) are NB consecutive bytes
-        uint8_t* brow = bp_buf(X, it) + static_cast<size_t>(t + 1) * G + tm.a_out_index(0, 0);
-        uint64_t packed = 0;
+        // the thread's groups a_out_index(u, bb) are NB consecutive groups: NB * KB bits
+        uint8_t* brow = bp_buf(X, it) + static_cast<size_t>(t + 1) * row_bytes + ((tm.a_out_index(0, 0) * KB) >> 3);
+        uint32_t packed = 0;
 #pragma unroll
-        for (int v = 0; v < NB; ++v)
-          packed |= static_cast<uint64_t>(static_cast<uint8_t>(bj[X][v / BT][v % BT])) << (8 * v);
-        if constexpr (NB == 8) {
-          *reinterpret_cast<uint64_t*>(brow) = packed;
+        for (int v = 0; v < NB; ++v) packed |= static_cast<uint32_t>(bj[X][v / BT][v % BT]) << (KB * v);
+        if constexpr (NB * KB == 8) {
+          *brow = static_cast<uint8_t>(packed);
         } else {
-          *reinterpret_cast<uint32_t*>(brow) = static_cast<uint32_t>(packed);
+          *reinterpret_cast<uint16_t*>(brow) = static_cast<uint16_t>(packed);
         }
       }
       pipe.after_stores();
