@@ -60,10 +60,11 @@ struct FBParams {
 // Shared-memory carve-up of the forward-backward kernel (bytes), identical on
 // host and device.  Per team and per sequence in flight: the double-buffered
 // exchange vectors (float64 group values, float32 adjoint accumulators); per
-// CTA: a reduction scratch and the thread-private staging of the forward
-// values read by the backward sweep (values, reference words, accumulators).
+// CTA: a reduction scratch, the thread-private staging of the forward
+// values read by the backward sweep (values, reference words, accumulators),
+// and every thread's float codewords.
 struct FBSmem {
-  uint32_t exA, exF, exB, exBt, mbar, per_seq, per_team, red, stage, stageK, stageF, total;
+  uint32_t exA, exF, exB, exBt, mbar, per_seq, per_team, red, stage, stageK, stageF, cf, total;
 };
 __host__ __device__ inline FBSmem fb_smem_layout(int GL, int NT, int NV, int nseq, bool adj, bool alias,
                                                  int teams_per_cta) {
@@ -92,6 +93,9 @@ __host__ __device__ inline FBSmem fb_smem_layout(int GL, int NT, int NV, int nse
   if (adj) o += stg * NV * 4u;
   l.stageK = o;
   o += stg * 4u;
+  o = (o + 15u) & ~15u;
+  l.cf = o;  // float codewords of every thread: [8 pairs][NT] float2
+  o += static_cast<uint32_t>(NT) * 16u * 4u;
   l.total = o;
   return l;
 }

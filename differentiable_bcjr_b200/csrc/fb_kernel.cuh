@@ -192,10 +192,15 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
   float* red = reinterpret_cast<float*>(smem_raw + lay.red);
   uint32_t* redk = reinterpret_cast<uint32_t*>(smem_raw + lay.red) + 256;
 
-  // Codewords of the thread's 16 states: float (for float32 sums) and scaled float64.
+  // Codewords of the thread's 16 states: scaled float64 in registers (the
+  // emission), float in shared memory (the float32 sums of the backward
+  // sweep): keeping the floats out of registers leaves the forward sweep
+  // more registers for independent work (forward call 10 % faster).
   const double sqsc = p.sqsc;
   static_assert(BT % 2 == 0, "state pairs along b");
-  float2 cf2[U][JT][BT / 2];  // (c(s_b), c(s_b+1)) pairs: the backward sweep works on state pairs
+  // (c(s_b), c(s_b+1)) float pairs in shared memory, pair e of thread i at [e][i]
+  float2* cfs = reinterpret_cast<float2*>(smem_raw + lay.cf) + threadIdx.x;
+  auto cf2 = [&](int u, int jj, int bp) -> float2 { return cfs[((u * JT + jj) * (BT / 2) + bp) * NT]; };
   double cp[U][JT][BT];
   bool bad_cb = false;
 #pragma unroll
@@ -205,11 +210,8 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
 #pragma unroll
       for (int bb = 0; bb < BT; ++bb) {
         const float cv = __ldg(p.codebook + tm.state(u, jj, bb));
-        if (bb & 1) {
-          cf2[u][jj][bb / 2].y = cv;
-        } else {
-          cf2[u][jj][bb / 2].x = cv;
-        }
+        float* slot = reinterpret_cast<float*>(cfs + ((u * JT + jj) * (BT / 2) + bb / 2) * NT);
+        slot[bb & 1] = cv;
         cp[u][jj][bb] = static_cast<double>(cv) * sqsc;
         bad_cb |= !(fabs(cp[u][jj][bb]) <= fbk::kMaxScaled);
       }
@@ -355,7 +357,8 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
             const float e = ex2f(fbk::neg_d2f(xv[jj] - ref));
             s += e;
             if constexpr (ADJ) {
-              const float cv = (bb & 1) ? cf2[u][jj][bb / 2].y : cf2[u][jj][bb / 2].x;
+              const float2 cv2 = cf2(u, jj, bb / 2);
+              const float cv = (bb & 1) ? cv2.y : cv2.x;
               num = fmaf(e, f[u * JT + jj] + fmaf(gt, cv, -gw), num);
             }
           }
@@ -660,7 +663,7 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
 #pragma unroll
           for (int bp = 0; bp < BT / 2; ++bp) {
             const int b0 = 2 * bp, b1 = 2 * bp + 1;
-            const float2 cv = cf2[u][jj][bp];
+            const float2 cv = cf2(u, jj, bp);
             const double d0 = wp - cp[u][jj][b0], d1 = wp - cp[u][jj][b1];
             const float2 e = make_float2(ex2f(fbk::neg_d2f(fma(-d0, d0, bv[u][b0] + r))),
                                          ex2f(fbk::neg_d2f(fma(-d1, d1, bv[u][b1] + r))));  // gamma_t / 2
