@@ -26,6 +26,7 @@ import os
 import re
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -85,7 +86,9 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        # raw samples go to BCJR_CLOCKS_DIR (default: the system temporary directory)
+        out_dir = os.environ.get("BCJR_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(out_dir, f"bcjr_clocks_rank{gpu_index}_{os.getpid()}.csv")
 
     def start(self):
         try:
