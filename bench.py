@@ -208,9 +208,9 @@ def load_peaks():
 
 
 # Sources that define each measured kernel (its ncu counters go stale when they change).
-FB_SOURCES = ("fb_", "bcjr_device", "team", "bcjr_internal")
-VITERBI_SOURCES = ("viterbi_kernel", "bitshift_kernels", "bcjr_device", "team", "bcjr_internal")
-DENSE_SOURCES = ("dense_kernel", "bcjr_device", "bcjr_internal")
+FB_SOURCES = ("fb_", "bcjr_device", "team", "bcjr_internal", "bcjr_common")
+VITERBI_SOURCES = ("viterbi_kernel", "bitshift_kernels", "bcjr_device", "team", "bcjr_internal", "bcjr_common")
+DENSE_SOURCES = ("dense_kernel", "dense_internal", "bcjr_device", "bcjr_common")
 
 
 def kernel_source_hash(prefixes=FB_SOURCES):

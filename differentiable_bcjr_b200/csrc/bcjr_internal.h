@@ -4,13 +4,11 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "bcjr_common.h"
+
 namespace bcjr {
 
-// Device-side error bits, OR-ed into the status word at the head of the workspace.
-enum : int {
-  kDevNonFinite = 1,   // log Z (or a Viterbi metric) came out NaN or infinite
-  kDevTimeout = 2,     // a bounded wait gave up (the results of the call are not valid)
-};
+
 
 // Geometry of one launch over the bitshift trellis (host-computed).
 struct TeamGeometry {
@@ -113,68 +111,9 @@ struct ViterbiParams {
   int num_slots;
 };
 
-// Dense (fully connected) trellis: 256 states, 32 sequences per CTA.
-constexpr int kDenseStates = 256;
-constexpr int kDenseRows = 32;
-
-struct DenseParams {
-  const float* w;          // [N][n]
-  const float* codebook;   // [S]
-  const float* g;          // [N][n] upstream gradient (backward)
-  const float* what_in;    // [N][n] soft codeword of the forward call (backward; centring)
-  float* w_hat;            // [N][n] (forward)
-  float* marginals;        // [N][n][S] or null (forward)
-  float* log_z;            // [N] or null (forward)
-  float* grad_w;           // [N][n] (backward)
-  float* gc_part;          // [grid][S] per-CTA codebook-gradient partials (backward)
-  const float* P;          // [S][S] exp(Lambda)
-  const float* PT;         // [S][S] its transpose
-  float* ckx;              // per CTA [n][32][S] normalised forward vectors
-  float* ckf;              // per CTA [n][32][S] forward adjoint accumulators (backward)
-  float* ckv;              // per CTA [n][32][S] rows V of the log-transition gradient, or null
-  float* ckw;              // per CTA [n][32][S] rows W of the log-transition gradient (with ckv)
-  float* mtab;             // per CTA [n][32] emission reference of each step
-  int* status;
-  size_t ck_stride;        // floats per CTA in ckx / ckf
-  size_t mt_stride;        // floats per CTA in mtab
-  float sc2;               // log2(e) / T
-  float two_over_T;
-  int n, N;
-};
-
-// Log-transition gradient of the dense trellis (dense_dlam_kernel.cu): rows of
-// X, U, V, W written by the backward kernel, one region per backward CTA
-// (`region_stride` floats apart), `spr` stages of 8 rows per region.
-struct DlamParams {
-  const float* X;
-  const float* U;
-  const float* V;
-  const float* W;
-  float* part;             // [grid][S][S] per-CTA partial sums
-  int* status;
-  long long region_stride;
-  long long spr;
-  long long total_stages;
-};
-
-// Dense launchers (dense_kernel.cu, dense_dlam_kernel.cu).
-size_t dense_smem_bytes(bool adjoint);
-cudaError_t dense_geometry(bool adjoint, int n_seq, int* grid);
-int dense_max_grid(bool adjoint);
-cudaError_t launch_dense_prep(const float* lam, const DenseParams& p, cudaStream_t s);
-cudaError_t launch_dense(const DenseParams& p, const float* lam, bool adjoint, int grid, cudaStream_t s,
-                         bool prep = true);
-size_t dlam_smem_bytes();
-cudaError_t dlam_grid(long long total_stages, int* grid);
-cudaError_t launch_dlam(const DlamParams& p, int grid, cudaStream_t s);
-cudaError_t launch_dlam_reduce(const float* part, int nparts, const float* P, float* out, int accumulate,
-                               cudaStream_t s);
-
 // Launchers (bitshift_kernels.cu).  Return a cudaError_t from the launch.
 cudaError_t launch_fb(const FBParams& p, const TeamGeometry& g, bool adjoint, cudaStream_t s);
 cudaError_t launch_viterbi(const ViterbiParams& p, const TeamGeometry& g, cudaStream_t s);
-cudaError_t launch_gradc_reduce(const float* gc_part, int num_slots, int S, float* grad_c,
-                                int accumulate, cudaStream_t s);
 // Host-side geometry and persistent grid for this device.  cudaErrorNotSupported
 // when no configuration fits the shared memory of one CTA.
 cudaError_t fb_geometry(int L, int k, int n_seq, bool adjoint, int C, int nseq_request, TeamGeometry* g);

@@ -5,7 +5,7 @@
 #include <cstdint>
 
 #include "bcjr.h"
-#include "bcjr_internal.h"
+#include "dense_internal.h"
 
 namespace {
 

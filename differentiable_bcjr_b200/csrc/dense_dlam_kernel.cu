@@ -35,7 +35,7 @@
 #include <cstdint>
 
 #include "bcjr_device.cuh"
-#include "bcjr_internal.h"
+#include "dense_internal.h"
 
 namespace bcjr {
 namespace dlam {

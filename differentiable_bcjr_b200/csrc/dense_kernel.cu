@@ -34,7 +34,7 @@
 #include <cmath>
 
 #include "bcjr_device.cuh"
-#include "bcjr_internal.h"
+#include "dense_internal.h"
 
 namespace bcjr {
 namespace dense {
