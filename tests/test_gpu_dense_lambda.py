@@ -163,3 +163,11 @@ def test_log_transition_gradient_accumulates(B):
     torch.cuda.synchronize()
     torch.testing.assert_close(gc, gc1 + 0.25, rtol=0, atol=1e-6)
     torch.testing.assert_close(gl, gl1 - 0.5, rtol=0, atol=1e-6)
+
+
+def test_log_transition_gradient_empty_batch(B):
+    c, _, _, lam = _case(5, 1, seed=7)
+    w0 = torch.empty((0, 5), device="cuda")
+    gw, gc, gl = B.bcjr_dense_backward(w0, w0, c.cuda(), lam.cuda(), w0, 0.3, want_grad_log_trans=True)
+    torch.cuda.synchronize()
+    assert gw.numel() == 0 and bool((gc == 0).all()) and bool((gl == 0).all())
