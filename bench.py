@@ -561,7 +561,7 @@ def run_dense(args):
                              "frac": flops_f / fwd_s / fp32_peak},
             "kernels_ms": {"bcjr_dense_forward": 1e3 * fwd_s,
                            ("bcjr_dense_backward_lambda" if wl else "bcjr_dense_backward"): 1e3 * bwd_s},
-            "gpu_launches": (8 if wl else 5) * args.steps,
+            "gpu_launches": (7 if wl else 5) * args.steps,  # prep + forward; prep + adjoint + reduction (+ tensor-core sum + reduction)
             "clocks": clocks,
         }
         if wl:
