@@ -60,9 +60,10 @@ def parse():
     ap.add_argument("--checkpoint-interval", type=int, default=1)
     ap.add_argument("--n-seq", type=int, default=0,
                     help="sequences per GPU (default: the workload's 65536); smaller only for profiling")
-    ap.add_argument("--workload", default="projection", choices=["projection", "dense", "viterbi"],
+    ap.add_argument("--workload", default="projection", choices=["projection", "dense", "viterbi", "bitwidth"],
                     help="projection: the S=2^16, k=2 headline; dense: the 256-state fully connected trellis; "
-                         "viterbi: hard decode of the projection")
+                         "viterbi: hard decode of the projection; bitwidth: k = 2, 3, 4 at S=2^16 on "
+                         "16384 sequences (forward, backward and hard decode per k)")
     ap.add_argument("--with-lambda", action="store_true",
                     help="dense workload: the backward call also returns dL/dLambda (tensor-core reduction)")
     return ap.parse_args()
@@ -707,6 +708,65 @@ def run_viterbi(args):
     return 0
 
 
+# --------------------------------------------------------------------------
+# Bit-width sweep: k = 2, 3, 4 at S = 2^16 (one GPU)
+# --------------------------------------------------------------------------
+def run_bitwidth(args):
+    world, rank, local = dist_env()
+    if world > 1:
+        raise SystemExit("--workload bitwidth runs on one GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import differentiable_bcjr_b200 as B
+
+    W = I.WORKLOADS["bitwidth_L16_k234"]
+    L, n, N, T = W["state_bits"], W["seq_len"], W["n_seq"], W["T"][0]
+    if args.n_seq > 0:
+        N = args.n_seq
+    S = 1 << L
+    c, w, g = I.codebook(S).to(dev), I.weights(N, n).to(dev), I.upstream_grad(N, n).to(dev)
+    stream = torch.cuda.current_stream(dev)
+    peaks = load_peaks()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    max_mhz = float(peaks.get("sm_max_mhz", 1965.0))
+    mufu_peak = MUFU_OPS_PER_CLK_PER_SM * sms * max_mhz * 1e6
+    sampler = ClockSampler(local)
+    sampler.start()
+    per_k = {}
+    for k in W["k"]:
+        ws_f, ws_b, ws_v = B.Workspace(dev), B.Workspace(dev), B.Workspace(dev)
+        times = []
+        for it in range(args.warmup + args.steps):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            torch.cuda.synchronize(dev)
+            ev[0].record(stream)
+            wh, _, _ = B.bcjr_forward(w, c, T, L, k, ws=ws_f)
+            ev[1].record(stream)
+            B.bcjr_backward(g, w, c, wh, T, L, k, ws=ws_b)
+            ev[2].record(stream)
+            B.viterbi_decode(w, c, L, k, ws=ws_v)
+            ev[3].record(stream)
+            torch.cuda.synchronize(dev)
+            if it >= args.warmup:
+                times.append([ev[i].elapsed_time(ev[i + 1]) for i in range(3)])
+        f, b, v = (statistics.mean(x[i] for x in times) for i in range(3))
+        per_k[str(k)] = {"bcjr_forward_ms": f, "bcjr_backward_ms": b, "viterbi_decode_ms": v,
+                         "fwd_bwd_weights_per_s": N * n / ((f + b) / 1e3),
+                         "exp_roofline_frac": ALG_MUFU_PER_STATE_STEP * N * n * S / ((f + b) / 1e3) / mufu_peak}
+    clocks = sampler.stop()
+    k2 = per_k["2"]
+    line = {"metric": "BCJR fwd+bwd weights/s at S=2^16 for k = 2, 3, 4 (16384 sequences); % of exp-pipe peak",
+            "value": k2["fwd_bwd_weights_per_s"], "unit": "weights/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": k2["bcjr_forward_ms"] + k2["bcjr_backward_ms"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "bitwidth_L16_k234", "state_bits": L, "k": W["k"], "seq_len": n,
+                       "n_seq_per_gpu": N, "T": T,
+                       "l2": "no flush: each call streams > 1 GiB of workspace, larger than the 126 MB L2"},
+            "per_k": per_k, "gpu_launches": 4 * len(W["k"]) * args.steps, "clocks": clocks}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -715,6 +775,8 @@ def main():
         return run_dense(args)
     if args.workload == "viterbi":
         return run_viterbi(args)
+    if args.workload == "bitwidth":
+        return run_bitwidth(args)
     return run_gpu(args)
 
 
