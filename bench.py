@@ -686,7 +686,7 @@ def run_viterbi(args):
                          "kernel": "viterbi_kernel (viterbi_decode)",
                          "peak_source": f"{FP64_OPS_PER_CLK_PER_SM} fp64 lanes/clk/SM x {sms} SMs x {max_mhz:.0f} MHz"},
             "kernels_ms": {"viterbi_decode": ms_per_step},
-            "gpu_launches": args.steps,
+            "gpu_launches": 2 * args.steps,  # decode + hard-codeword gather
             "clocks": clocks,
         }
         if e2e is not None:

@@ -30,6 +30,13 @@ __global__ void gradc_reduce_kernel(const float* __restrict__ part, int num_slot
   out[s] = accumulate ? out[s] + acc : acc;
 }
 
+// w_hard[i] = codebook[states[i]]: the hard codeword of every decoded state.
+__global__ void gather_codewords_kernel(const int32_t* __restrict__ states, const float* __restrict__ codebook,
+                                        float* __restrict__ w_hard, size_t total) {
+  const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < total) w_hard[i] = __ldg(codebook + __ldg(states + i));
+}
+
 // ---------------------------------------------------------------------------
 // Host side: geometry and launches.
 // ---------------------------------------------------------------------------
@@ -266,7 +273,16 @@ cudaError_t launch_viterbi(const ViterbiParams& p, const TeamGeometry& g, cudaSt
   if (!fn) return cudaErrorNotSupported;
   ViterbiParams copy = p;
   void* args[] = {&copy};
-  return launch(fn, g, args, s);
+  cudaError_t e = launch(fn, g, args, s);
+  if (e != cudaSuccess || !p.w_hard) return e;
+  // The hard codewords are gathered after the decode: inside it, the walker's
+  // codebook load would hold up its whole warp, and with it the cluster's step.
+  const size_t total = static_cast<size_t>(p.N) * p.n;
+  if (total == 0) return cudaSuccess;
+  const int threads = 256;
+  const unsigned blocks = static_cast<unsigned>((total + threads - 1) / threads);
+  gather_codewords_kernel<<<blocks, threads, 0, s>>>(p.states, p.codebook, p.w_hard, total);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_gradc_reduce(const float* gc_part, int num_slots, int S, float* grad_c, int accumulate,

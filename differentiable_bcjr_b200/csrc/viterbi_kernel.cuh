@@ -127,7 +127,6 @@ __global__ void __launch_bounds__(NTB, 1) viterbi_kernel(const ViterbiParams p) 
   auto walk_step = [&](int x, int ti) {
     if (ti < n - 1) wk_s[x] = (wk_j[x] << (L - k)) | (wk_s[x] >> k);
     p.states[static_cast<size_t>(wk_seq[x]) * n + ti] = wk_s[x];
-    if (p.w_hard) p.w_hard[static_cast<size_t>(wk_seq[x]) * n + ti] = __ldg(p.codebook + wk_s[x]);
     if (ti >= 1) {
       const int bit = (wk_s[x] >> k) * KB;
       wk_j[x] = (wk_bp[x][static_cast<size_t>(ti) * row_bytes + (bit >> 3)] >> (bit & 7)) & (K - 1);
