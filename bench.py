@@ -52,7 +52,7 @@ ALG_MUFU_PER_STATE_STEP = 4       # one forward and one backward log-sum-exp in 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=4)
+    ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -60,10 +60,12 @@ def parse():
     ap.add_argument("--checkpoint-interval", type=int, default=1)
     ap.add_argument("--n-seq", type=int, default=0,
                     help="sequences per GPU (default: the workload's 65536); smaller only for profiling")
-    ap.add_argument("--workload", default="projection", choices=["projection", "dense", "viterbi", "bitwidth"],
+    ap.add_argument("--workload", default="projection",
+                    choices=["projection", "dense", "viterbi", "bitwidth", "mufu"],
                     help="projection: the S=2^16, k=2 headline; dense: the 256-state fully connected trellis; "
                          "viterbi: hard decode of the projection; bitwidth: k = 2, 3, 4 at S=2^16 on "
-                         "16384 sequences (forward, backward and hard decode per k)")
+                         "16384 sequences (forward, backward and hard decode per k); mufu: throughput of the "
+                         "ex2/lg2 pipe (the roofline's peak)")
     ap.add_argument("--with-lambda", action="store_true",
                     help="dense workload: the backward call also returns dL/dLambda (tensor-core reduction)")
     return ap.parse_args()
@@ -252,7 +254,8 @@ def run_gpu(args):
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    import differentiable_bcjr_b200 as B
+    import differentiable_bcjr_b200 as B  # noqa: F401  (fails loudly without the CUDA library)
+    from differentiable_bcjr_b200 import distributed as D
 
     W = I.WORKLOADS[WORKLOAD]
     L, k, n, N, temps = W["state_bits"], W["k"], W["seq_len"], W["n_seq"], W["T"]
@@ -260,7 +263,12 @@ def run_gpu(args):
         N = args.n_seq
     S = 1 << L
     C = args.checkpoint_interval
-    # each rank: its own projection matrix (seed offset by rank), shared codebook
+    # Weak scaling: the global batch is `world` projection matrices stacked
+    # (world * N sequences); this rank owns its block of rows (shard_bounds),
+    # which is the projection drawn with the rank's own seed.  The codebook is
+    # shared and its gradient is summed over ranks (ShardedSoftQuant).
+    lo, hi = D.shard_bounds(world * N, world, rank)
+    assert hi - lo == N
     c_h = I.codebook(S)
     w_h = I.weights(N, n, seed=I.SEED_WEIGHTS + 100 * rank)
     g_h = I.upstream_grad(N, n, seed=I.SEED_UPSTREAM + 100 * rank)
@@ -268,19 +276,13 @@ def run_gpu(args):
     w = w_h.to(dev)
     g = g_h.to(dev)
     w_hat = torch.empty_like(w)
-    grad_c = torch.zeros(S, device=dev)
-    ws_f = B.Workspace(dev)
-    ws_b = B.Workspace(dev)
+    sq = D.ShardedSoftQuant(c, L, k, checkpoint_interval=C)
     stream = torch.cuda.current_stream(dev)
 
     def step(i, w_in, g_in, what_out):
         T = temps[i % len(temps)]
-        B.bcjr_forward(w_in, c, T, L, k, checkpoint_interval=C, ws=ws_f, out=what_out)
-        gw, gc = B.bcjr_backward(g_in, w_in, c, what_out, T, L, k, checkpoint_interval=C, ws=ws_b,
-                                 grad_codebook=grad_c, accumulate_codebook=False)
-        if world > 1:
-            torch.distributed.all_reduce(gc)
-        return gw, gc
+        sq.forward(w_in, T, out=what_out)
+        return sq.backward(g_in, w_in, what_out, T)
 
     def barrier():
         if world > 1:
@@ -303,23 +305,17 @@ def run_gpu(args):
     for i in range(args.steps):
         T = temps[i % len(temps)]
         ev[i][0].record(stream)
-        B.bcjr_forward(w, c, T, L, k, checkpoint_interval=C, ws=ws_f, out=w_hat)
+        sq.forward(w, T, out=w_hat)
         ev[i][1].record(stream)
-        gw, gc = B.bcjr_backward(g, w, c, w_hat, T, L, k, checkpoint_interval=C, ws=ws_b,
-                                 grad_codebook=grad_c, accumulate_codebook=False)
+        gw, gc = sq.backward(g, w, w_hat, T)  # + the all-reduce of grad_codebook on several ranks
         ev[i][2].record(stream)
-        if world > 1:
-            torch.distributed.all_reduce(gc)
     end.record(stream)
     barrier()
     clocks = sampler.stop()
-    elapsed_ms = start.elapsed_time(end)
+    elapsed_ms = D.max_over_ranks(start.elapsed_time(end), dev)
     fwd_ms = [a.elapsed_time(b) for a, b, _ in ev]
     bwd_ms = [b.elapsed_time(cc) for _, b, cc in ev]
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    step_med_ms = D.max_over_ranks(statistics.median(f + b for f, b in zip(fwd_ms, bwd_ms)), dev)
     ms_per_step = elapsed_ms / args.steps
     weights_total = world * N * n
     value = weights_total / (ms_per_step / 1e3)
@@ -349,11 +345,7 @@ def run_gpu(args):
             gc_pin.copy_(gc, non_blocking=True)
         e2.record(stream)
         barrier()
-        e2e_ms = s2.elapsed_time(e2)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = D.max_over_ranks(s2.elapsed_time(e2), dev)
         e2e = {"value": weights_total / (e2e_ms / args.steps / 1e3), "unit": "weights/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps}
 
@@ -362,27 +354,31 @@ def run_gpu(args):
         props = torch.cuda.get_device_properties(dev)
         sms = props.multi_processor_count
         max_mhz = float(peaks.get("sm_max_mhz", 1965.0))
-        mufu_peak = MUFU_OPS_PER_CLK_PER_SM * sms * max_mhz * 1e6          # ops/s at the max clock
+        # the MUFU peak at the clock the timed region ran at (median of the samples)
+        run_mhz = float(clocks["sm_mhz"]) if clocks and clocks.get("sm_mhz") else max_mhz
+        mufu_peak = MUFU_OPS_PER_CLK_PER_SM * sms * run_mhz * 1e6          # ops/s
         state_steps = N * n * S
-        # dominant kernel: the backward launch (2 log-sum-exp sweeps per state-step)
-        bwd_avg_s = statistics.mean(bwd_ms) / 1e3
-        fwd_avg_s = statistics.mean(fwd_ms) / 1e3
-        achieved = 2 * state_steps / bwd_avg_s
+        # dominant kernel: the backward launch (2 log-sum-exp sweeps per state-step), median over steps
+        bwd_med_s = statistics.median(bwd_ms) / 1e3
+        fwd_med_s = statistics.median(fwd_ms) / 1e3
+        achieved = 2 * state_steps / bwd_med_s
         traffic = scaled_traffic(load_traffic().get("bwd_dram_bytes_per_launch"), N, I.WORKLOADS[WORKLOAD]["n_seq"])
-        frac_total = ALG_MUFU_PER_STATE_STEP * state_steps * world / (ms_per_step / 1e3) / (mufu_peak * world)
+        frac_total = ALG_MUFU_PER_STATE_STEP * state_steps / (step_med_ms / 1e3) / mufu_peak
         line = {
             "metric": METRIC, "value": value, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": _config(world, C, N),
             "state_updates_per_s": value * S,
+            "step_ms_median": step_med_ms,
             "exp_roofline_frac": frac_total,
             "roofline": {"bound": "alu", "pipe": "MUFU (ex2/lg2)", "achieved": achieved / 1e12,
                          "peak": mufu_peak / 1e12, "unit": "Texp/s", "frac": achieved / mufu_peak,
                          "traffic": traffic, "kernel": "fb_kernel<adjoint> (bcjr_backward)",
-                         "peak_source": f"{MUFU_OPS_PER_CLK_PER_SM} ops/clk/SM x {sms} SMs x {max_mhz:.0f} MHz "
-                                        "(sm_max_mhz of MEASURED_PEAKS.json)"},
-            "kernels_ms": {"bcjr_forward": 1e3 * fwd_avg_s, "bcjr_backward": 1e3 * bwd_avg_s},
+                         "peak_source": f"{MUFU_OPS_PER_CLK_PER_SM} ops/clk/SM (measured: bench.py --workload mufu) "
+                                        f"x {sms} SMs x {run_mhz:.0f} MHz (median SM clock of the timed region)"},
+            "kernels_ms": {"bcjr_forward": 1e3 * fwd_med_s, "bcjr_backward": 1e3 * bwd_med_s,
+                           "statistic": f"median of {args.steps} steps"},
             "gpu_launches": 3 * args.steps,
             "clocks": clocks,
         }
@@ -402,6 +398,33 @@ def run_gpu(args):
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
+    return 0
+
+
+# --------------------------------------------------------------------------
+# Special-function pipe throughput (the exp-pipe roofline's denominator)
+# --------------------------------------------------------------------------
+def run_mufu(args):
+    world, rank, local = dist_env()
+    if rank != 0:
+        return 0
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import differentiable_bcjr_b200 as B
+    iters = 4096
+    for _ in range(max(args.warmup, 1)):
+        B.probe_xu("ex2", iters, dev)
+    res = {op: [B.probe_xu(op, iters, dev) for _ in range(max(args.steps, 1))] for op in ("ex2", "lg2")}
+    per = {op: statistics.median(r["ops_per_clk_per_sm"] for r in rs) for op, rs in res.items()}
+    line = {"metric": "special-function pipe throughput, ex2.approx.ftz.f32 and lg2.approx.ftz.f32",
+            "value": per["ex2"], "unit": "ops/clk/SM", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "higher_is_better": True, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "xu_probe", "ctas": res["ex2"][0]["sms"], "threads_per_cta": 1024,
+                       "chains_per_thread": 16, "iters": iters},
+            "ex2_ops_per_clk_per_sm": per["ex2"], "lg2_ops_per_clk_per_sm": per["lg2"],
+            "spread_over_sms": {op: [rs[0]["min"], rs[0]["max"]] for op, rs in res.items()},
+            "gpu_launches": 2 * max(args.steps, 1) + max(args.warmup, 1)}
+    print(json.dumps(line), flush=True)
     return 0
 
 
@@ -777,6 +800,8 @@ def main():
         return run_viterbi(args)
     if args.workload == "bitwidth":
         return run_bitwidth(args)
+    if args.workload == "mufu":
+        return run_mufu(args)
     return run_gpu(args)
 
 

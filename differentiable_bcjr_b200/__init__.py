@@ -24,7 +24,7 @@ __all__ = [
     "LIB_PATH", "lib", "BCJRError", "bcjr_forward", "bcjr_backward", "viterbi_decode",
     "bcjr_dense_forward", "bcjr_dense_backward", "workspace_size", "Workspace",
     "SoftTrellisQuant", "soft_quantize", "DenseTrellisQuant", "dense_soft_quantize", "bcjr_forward_static_scratch",
-    "OP_FORWARD", "OP_BACKWARD", "OP_VITERBI",
+    "static_scratch_status", "probe_xu", "OP_FORWARD", "OP_BACKWARD", "OP_VITERBI",
     "OP_DENSE_FORWARD", "OP_DENSE_BACKWARD", "OP_DENSE_BACKWARD_LAMBDA", "STATUS",
 ]
 
@@ -43,7 +43,7 @@ class BCJRError(RuntimeError):
 
 class Options(ctypes.Structure):
     _fields_ = [("checkpoint_interval", ctypes.c_int), ("sequences_in_flight", ctypes.c_int),
-                ("reserved", ctypes.c_int * 6)]
+                ("timeout_probe_cycles", ctypes.c_int), ("reserved", ctypes.c_int * 5)]
 
 
 _lib = None
@@ -65,7 +65,9 @@ _SIGS = {
     "bcjr_dense_backward_lambda": (_I, [_P, _P, _P, _P, _P, _F, _I, _I, _I, _P, _P, _P, _I,
                                         ctypes.POINTER(Options), _P, _Z, _P]),
     "bcjr_get_status": (_I, [_P, _P]),
+    "bcjr_static_scratch_status": (_I, [_P]),
     "bcjr_status_string": (ctypes.c_char_p, [_I]),
+    "bcjr_probe_xu": (_I, [_I, _I, _P, _P, _I, _P]),
     "bcjr_version": (_I, []),
 }
 
@@ -85,10 +87,11 @@ def lib():
     return _lib
 
 
-def _opts(checkpoint_interval: int = 0, sequences_in_flight: int = 0):
+def _opts(checkpoint_interval: int = 0, sequences_in_flight: int = 0, timeout_probe_cycles: int = 0):
     o = Options()
     o.checkpoint_interval = int(checkpoint_interval)
     o.sequences_in_flight = int(sequences_in_flight)
+    o.timeout_probe_cycles = int(timeout_probe_cycles)
     return o
 
 
@@ -149,9 +152,10 @@ def get_status(ws_tensor: torch.Tensor) -> int:
 
 
 def bcjr_forward(w, codebook, T, state_bits, k, want_marginals=False, checkpoint_interval=0, ws=None,
-                 out=None, sequences_in_flight=0):
+                 out=None, sequences_in_flight=0, timeout_probe_cycles=0):
     """Soft codeword of every row of w [N][n] (float32, CUDA).  Returns
-    (w_hat [N][n], marginals [N][n][S] or None, log_z [N])."""
+    (w_hat [N][n], marginals [N][n][S] or None, log_z [N]).
+    `timeout_probe_cycles` is the testing aid of bcjr_options (see bcjr.h)."""
     _need_cuda(w, codebook)
     N, n = w.shape
     S = 1 << state_bits
@@ -159,7 +163,7 @@ def bcjr_forward(w, codebook, T, state_bits, k, want_marginals=False, checkpoint
     w_hat = out if out is not None else torch.empty((N, n), dtype=torch.float32, device=dev)
     marg = torch.empty((N, n, S), dtype=torch.float32, device=dev) if want_marginals else None
     log_z = torch.empty((N,), dtype=torch.float32, device=dev)
-    o = _opts(checkpoint_interval, sequences_in_flight)
+    o = _opts(checkpoint_interval, sequences_in_flight, timeout_probe_cycles)
     nbytes = lib().bcjr_workspace_size(OP_FORWARD, state_bits, k, n, N, ctypes.byref(o))
     if nbytes == 0:
         raise BCJRError(2, "bcjr_workspace_size")
@@ -173,18 +177,49 @@ def bcjr_forward(w, codebook, T, state_bits, k, want_marginals=False, checkpoint
 STATIC_SCRATCH_BYTES = 32 << 20
 
 
+def _expect(t, name, shape, dtype, device):
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, not {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, not {t.dtype}")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the weights on {device}")
+
+
 def bcjr_forward_static_scratch(w, codebook, T, state_bits, k, w_hat, log_z=None, marginals=None,
                                 checkpoint_interval=0):
     """bcjr_forward into caller-provided outputs, with the library's static
     device scratch as workspace: neither this function nor the library
     allocates device memory.  Calls on one device share that scratch, so they
-    must not overlap in time."""
+    must not overlap in time.  Every tensor must sit on w's device, which is
+    made current for the call."""
     _need_cuda(w, codebook, w_hat, log_z, marginals)
+    if w.dim() != 2:
+        raise ValueError("w must be [n_seq][seq_len]")
     N, n = w.shape
+    S = 1 << int(state_bits)
+    dev = w.device
+    _expect(w, "w", (N, n), torch.float32, dev)
+    _expect(codebook, "codebook", (S,), torch.float32, dev)
+    _expect(w_hat, "w_hat", (N, n), torch.float32, dev)
+    _expect(log_z, "log_z", (N,), torch.float32, dev)
+    _expect(marginals, "marginals", (N, n, S), torch.float32, dev)
     o = _opts(checkpoint_interval)
-    _check(lib().bcjr_forward_static_scratch(_ptr(w), _ptr(codebook), float(T), state_bits, k, n, N, _ptr(w_hat),
-                                             _ptr(marginals), _ptr(log_z), ctypes.byref(o), _stream(w.device)),
-           "bcjr_forward_static_scratch")
+    with torch.cuda.device(dev):
+        _check(lib().bcjr_forward_static_scratch(_ptr(w), _ptr(codebook), float(T), state_bits, k, n, N,
+                                                 _ptr(w_hat), _ptr(marginals), _ptr(log_z), ctypes.byref(o),
+                                                 _stream(dev)), "bcjr_forward_static_scratch")
+
+
+def static_scratch_status(device=None) -> int:
+    """Synchronise the current stream of `device` and return the device-side
+    status (a bcjr_status code) of the last bcjr_forward_static_scratch call
+    on that device."""
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        return int(lib().bcjr_static_scratch_status(_stream(dev)))
 
 
 def bcjr_backward(grad_w_hat, w, codebook, w_hat, T, state_bits, k, checkpoint_interval=0, ws=None,
@@ -337,3 +372,22 @@ class DenseTrellisQuant(torch.autograd.Function):
 
 def dense_soft_quantize(w, codebook, log_trans, T):
     return DenseTrellisQuant.apply(w, codebook, log_trans, T)
+
+
+def probe_xu(op: str = "ex2", iters: int = 4096, device=None) -> dict:
+    """Measured throughput of the special-function pipe (bcjr_probe.h): ex2
+    or lg2 instructions per clock per SM, from each CTA's own cycle count
+    (one CTA per SM).  Returns {"ops_per_clk_per_sm": median over SMs, "min",
+    "max", "sms", "ops"}."""
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    code = {"ex2": 0, "lg2": 1}[op]
+    sink = torch.empty(sms * 1024, dtype=torch.float32, device=dev)
+    cycles = torch.zeros(sms, dtype=torch.int64, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().bcjr_probe_xu(code, int(iters), _ptr(sink), _ptr(cycles), sms, _stream(dev)), "bcjr_probe_xu")
+        torch.cuda.synchronize(dev)
+    ops = 1024 * 16 * int(iters)
+    rates = sorted(ops / float(c) for c in cycles.cpu().tolist())
+    return {"ops_per_clk_per_sm": rates[len(rates) // 2], "min": rates[0], "max": rates[-1], "sms": sms,
+            "ops": ops * sms}

@@ -159,7 +159,7 @@ static bcjr_status fb_common(bool adjoint, const float* grad_w_hat, const float*
   bcjr_status st = check_trellis(L, k);
   if (st != BCJR_OK) return st;
   if (n < 1 || N < 0 || !(T > 0.f) || !std::isfinite(T)) return BCJR_ERR_INVALID_ARG;
-  if (opt && (opt->checkpoint_interval < 0 || opt->sequences_in_flight != 0))
+  if (opt && (opt->checkpoint_interval < 0 || opt->sequences_in_flight != 0 || opt->timeout_probe_cycles < 0))
     return BCJR_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int S = 1 << L;
@@ -211,8 +211,10 @@ static bcjr_status fb_common(bool adjoint, const float* grad_w_hat, const float*
   p.N = N;
   p.C = C;
   p.num_slots = g.num_slots;
+  p.probe_wait_cycles = opt ? opt->timeout_probe_cycles : 0;
   if ((st = reset_status(ws, s)) != BCJR_OK) return st;
   if ((st = from_cuda(bcjr::launch_fb(p, g, adjoint, s))) != BCJR_OK) return st;
+  if (p.probe_wait_cycles > 0 && g.cluster > 1) return BCJR_OK;  // the probe computed nothing
   if (adjoint) return from_cuda(bcjr::launch_gradc_reduce(p.gc_part, g.num_slots, S, grad_c, accumulate, s));
   return BCJR_OK;
 }

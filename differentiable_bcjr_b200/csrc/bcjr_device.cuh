@@ -217,10 +217,14 @@ __device__ __forceinline__ void mbar_arm(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
+// Bound of every device-side wait: about two seconds of SM clock.
+constexpr long long kWaitLimitCycles = 4000000000LL;
+
 // Wait for the phase with the given parity to complete (acquire at cluster
-// scope, so the other CTAs' st.async data is visible).  Gives up after about
-// two seconds of SM clock, ORs `timeout_bit` into *status and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, int timeout_bit) {
+// scope, so the other CTAs' st.async data is visible).  Gives up after
+// `limit` SM clock cycles, ORs `timeout_bit` into *status and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, int timeout_bit,
+                                          long long limit = kWaitLimitCycles) {
   const uint32_t a = smem_u32(bar);
   uint32_t done = 0;
   const long long t0 = clock64();
@@ -235,7 +239,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
         : "r"(a), "r"(parity), "r"(100000u)
         : "memory");
     if (done) return true;
-    if (clock64() - t0 > 4000000000LL) {
+    if (clock64() - t0 > limit) {
       atomicOr(status, timeout_bit);
       return false;
     }

@@ -53,6 +53,7 @@ struct FBParams {
   float two_over_T;
   int L, k, n, N, C;
   int num_slots;
+  long long probe_wait_cycles;  // > 0: only the bounded-wait probe runs (testing aid)
 };
 
 // Shared-memory carve-up of the forward-backward kernel (bytes), identical on

@@ -262,7 +262,16 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
 
   // Every CTA of the cluster must be running (and its mbarriers initialised)
   // before any of them writes into another's shared memory.
-  if constexpr (CL > 1) cluster_sync_all();
+  if constexpr (CL > 1) {
+    cluster_sync_all();
+    if (p.probe_wait_cycles > 0) {
+      // Testing aid: one bounded wait on a barrier nothing arrives at, before
+      // any exchange has started; it gives up and reports the timeout.
+      mbar_wait(mbar(0, 0, 0), 0u, p.status, kDevTimeout, p.probe_wait_cycles);
+      cluster_sync_all();
+      return;
+    }
+  }
 
   const int tvo = tm.tt * NV;  // this thread's offset in a thread-private row
   const int nsl = p.num_slots;

@@ -29,6 +29,9 @@ void* g_scratch_ptr[kMaxDevices] = {};
 
 // Address of this device's copy of the scratch, looked up once per device with
 // that device current.  The first lookup may load the module on the device.
+// The cached address belongs to the device's primary context: after
+// cudaDeviceReset the module is loaded anew and the address may change, so a
+// process that resets a device must not call these entry points on it again.
 bcjr_status scratch_for_current_device(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return BCJR_ERR_CUDA;
@@ -59,4 +62,12 @@ extern "C" bcjr_status bcjr_forward_static_scratch(const float* w, const float* 
   // before it is written.
   return bcjr_forward(w, codebook, T, state_bits, k, seq_len, n_seq, w_hat, marginals, log_z, opt, scratch,
                       BCJR_STATIC_SCRATCH_BYTES, stream);
+}
+
+extern "C" bcjr_status bcjr_static_scratch_status(bcjr_stream_t stream) {
+  void* scratch = nullptr;
+  const bcjr_status st = scratch_for_current_device(&scratch);
+  if (st != BCJR_OK) return st;
+  // The status word heads the scratch exactly as it heads a caller's workspace.
+  return bcjr_get_status(scratch, stream);
 }

@@ -63,7 +63,16 @@ typedef struct {
    * thread-block cluster when k >= 2, so that one sequence's step hides the
    * other's barrier, and one otherwise).  Other values are rejected. */
   int sequences_in_flight;
-  int reserved[6]; /* set to zero */
+  /* Testing aid for the bounded device-side waits; 0 in normal use.  When
+   * positive, a bcjr_forward / bcjr_backward call whose team is a
+   * thread-block cluster (state_bits >= 14) runs, before any exchange between
+   * the cluster's CTAs starts, one wait on an mbarrier that nothing arrives
+   * at, bounded at this many SM clock cycles; the wait gives up, the call
+   * computes nothing and bcjr_get_status then reports BCJR_ERR_TIMEOUT.  It
+   * exercises the same bounded wait and status path as the exchange, with
+   * nothing in flight.  Ignored by single-CTA teams and the other calls. */
+  int timeout_probe_cycles;
+  int reserved[5]; /* set to zero */
 } bcjr_options;
 
 typedef enum {
@@ -110,17 +119,34 @@ bcjr_status bcjr_forward(const float* w, const float* codebook, float T, int sta
  *    needs more than BCJR_STATIC_SCRATCH_BYTES, i.e. when
  *    bcjr_workspace_size(BCJR_OP_FORWARD, ...) is larger.
  *  - The device-side status word lives in the array and is cleared at the
- *    start of every call; a non-finite log-partition function shows as a
- *    non-finite log_z (bcjr_get_status cannot reach this scratch).
+ *    start of every call; read it with bcjr_static_scratch_status (below),
+ *    which reports BCJR_ERR_TIMEOUT or BCJR_ERR_NONFINITE from the last call
+ *    on the current device.
  *  - All calls on one device share the one array: two calls whose work
  *    overlaps in time (on different streams, or from several host threads
  *    without ordering) race on it and give wrong results.  Order them on one
  *    stream or with events.
+ *  - Footprint: every device that loads the library holds the 32 MiB array
+ *    until the process exits, whether or not it ever calls this entry point.
+ *    With the CUDA runtime's default lazy module loading that happens on the
+ *    first use of the library on the device; with CUDA_MODULE_LOADING=EAGER
+ *    at context creation.
+ *  - The address of the array is looked up once per device and cached for the
+ *    life of the process; a device reset (cudaDeviceReset) invalidates it, so
+ *    do not call this entry point on a device after resetting it.
+ *  - The calls use the current device: make the device that holds the
+ *    arguments current, and pass a stream of that device.
  */
 #define BCJR_STATIC_SCRATCH_BYTES (32u << 20) /* 32 MiB */
 bcjr_status bcjr_forward_static_scratch(const float* w, const float* codebook, float T, int state_bits,
                                         int k, int seq_len, int n_seq, float* w_hat, float* marginals,
                                         float* log_z, const bcjr_options* opt, bcjr_stream_t stream);
+
+/* Synchronise `stream` and return the device-side status of the most recent
+ * bcjr_forward_static_scratch call on the current device (BCJR_OK,
+ * BCJR_ERR_NONFINITE or BCJR_ERR_TIMEOUT), the counterpart of bcjr_get_status
+ * for the static scratch.  Allocates nothing. */
+bcjr_status bcjr_static_scratch_status(bcjr_stream_t stream);
 
 /*
  * Vector-Jacobian product of the soft codeword ("key technical innovations":

@@ -1,6 +1,7 @@
 """The C ABI library loads, exports what include/bcjr.h declares, and rejects
 bad arguments on the host before touching the GPU (CPU only)."""
 import ctypes
+import glob
 import os
 import re
 
@@ -8,6 +9,7 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "bcjr.h")
+HEADERS = sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
 @pytest.fixture(scope="module")
@@ -18,7 +20,7 @@ def lib():
 
 
 def declared_functions():
-    text = open(HEADER).read()
+    text = "\n".join(open(h).read() for h in HEADERS)
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)
     return sorted(set(names))
@@ -28,7 +30,8 @@ def test_header_declares_the_calls():
     names = declared_functions()
     for required in ["bcjr_forward", "bcjr_backward", "viterbi_decode", "bcjr_workspace_size",
                      "bcjr_get_status", "bcjr_status_string", "bcjr_dense_forward", "bcjr_dense_backward",
-                     "bcjr_dense_backward_lambda", "bcjr_forward_static_scratch"]:
+                     "bcjr_dense_backward_lambda", "bcjr_forward_static_scratch", "bcjr_static_scratch_status",
+                     "bcjr_probe_xu"]:
         assert required in names, names
 
 

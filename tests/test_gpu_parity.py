@@ -1,9 +1,11 @@
 """GPU parity with the float64 oracle through the C ABI (needs a B200).
 
 Shapes cover every kernel instantiation: k = 1..4, teams narrower than a
-warp (state_bits <= 8), single-CTA teams, and 2- and 4-CTA clusters
-(state_bits = 15, 16); ragged sequence lengths; checkpoint intervals C > 1
-that do and do not divide the length; the degenerate n = 1 and N = 0.
+warp (state_bits <= 8), single-CTA teams (state_bits 9..13, up to 512
+threads), and thread-block clusters of 2, 4 and 8 CTAs of 512 threads
+(state_bits = 14, 15, 16); ragged sequence lengths; checkpoint intervals
+C > 1 that do and do not divide the length; the degenerate n = 1 and N = 0;
+marginals of every team shape, clusters included.
 """
 import numpy as np
 import pytest
@@ -50,10 +52,10 @@ SHAPES = [
     (10, 1, 13, 2, 1.1),
     (11, 3, 9, 3, 0.25),
     (12, 4, 8, 2, 0.8),
-    (13, 2, 10, 2, 0.15),
-    (14, 3, 7, 2, 0.5),       # 1024-thread CTA
-    (15, 2, 6, 2, 0.35),      # 2-CTA cluster
-    (16, 2, 5, 2, 0.2),       # 4-CTA cluster
+    (13, 2, 10, 2, 0.15),     # 512-thread CTA
+    (14, 3, 7, 2, 0.5),       # 2-CTA cluster
+    (15, 2, 6, 2, 0.35),      # 4-CTA cluster
+    (16, 2, 5, 2, 0.2),       # 8-CTA cluster
     (16, 3, 4, 2, 0.1),
     (16, 4, 4, 2, 0.1),
 ]
@@ -71,6 +73,19 @@ def test_forward_backward_parity(B, L, k, n, N, T):
         assert_abs(marg, o_gamma, MARGINAL_ATOL, "marginals")
     assert_rel_l2(grad_w, o_gw, GRAD_REL_L2, "grad_w")
     assert_rel_l2(grad_c, o_gc, GRAD_REL_L2, "grad_codebook")
+
+
+@pytest.mark.parametrize("L,k,n,N,T", [(14, 2, 9, 2, 0.3), (15, 2, 12, 2, 0.2), (16, 2, 10, 2, 0.1),
+                                         (16, 2, 8, 3, 0.01), (16, 1, 6, 2, 0.4), (16, 3, 6, 2, 0.3),
+                                         (16, 4, 5, 2, 0.5), (15, 4, 7, 2, 0.25)])
+def test_cluster_team_marginals(B, L, k, n, N, T):
+    # the marginal-store instantiation of the 2-, 4- and 8-CTA cluster kernels
+    c, w, _ = _case(L, k, n, N, seed=600 + L * 5 + k)
+    w_hat, marg, log_z = B.bcjr_forward(w.cuda(), c.cuda(), T, L, k, want_marginals=True)
+    o_what, o_lz, o_gamma = oracle.forward(w, c, T, L, k, want_gamma=True)
+    assert_abs(marg, o_gamma, MARGINAL_ATOL, f"marginals L={L} k={k}")
+    assert_abs(w_hat, o_what, W_HAT_ATOL, f"w_hat L={L} k={k}")
+    np.testing.assert_allclose(to_np(log_z), o_lz, rtol=LOGZ_RTOL, atol=1e-4)
 
 
 @pytest.mark.parametrize("L,k,n,N,T,C", [(8, 2, 13, 3, 0.5, 4), (10, 3, 12, 2, 0.3, 3),
