@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--checkpoint-interval", type=int, default=1)
+    ap.add_argument("--seqs-in-flight", type=int, default=0,
+                    help="sequences a cluster team keeps in flight in the forward call (0: the library's choice)")
     ap.add_argument("--n-seq", type=int, default=0,
                     help="sequences per GPU (default: the workload's 65536); smaller only for profiling")
     ap.add_argument("--workload", default="projection",
@@ -276,7 +278,7 @@ def run_gpu(args):
     w = w_h.to(dev)
     g = g_h.to(dev)
     w_hat = torch.empty_like(w)
-    sq = D.ShardedSoftQuant(c, L, k, checkpoint_interval=C)
+    sq = D.ShardedSoftQuant(c, L, k, checkpoint_interval=C, sequences_in_flight=args.seqs_in_flight)
     stream = torch.cuda.current_stream(dev)
 
     def step(i, w_in, g_in, what_out):

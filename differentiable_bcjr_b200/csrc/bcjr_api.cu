@@ -159,7 +159,8 @@ static bcjr_status fb_common(bool adjoint, const float* grad_w_hat, const float*
   bcjr_status st = check_trellis(L, k);
   if (st != BCJR_OK) return st;
   if (n < 1 || N < 0 || !(T > 0.f) || !std::isfinite(T)) return BCJR_ERR_INVALID_ARG;
-  if (opt && (opt->checkpoint_interval < 0 || opt->sequences_in_flight != 0 || opt->timeout_probe_cycles < 0))
+  if (opt && (opt->checkpoint_interval < 0 || opt->sequences_in_flight < 0 || opt->sequences_in_flight > 4 ||
+              opt->timeout_probe_cycles < 0))
     return BCJR_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int S = 1 << L;
@@ -203,7 +204,8 @@ static bcjr_status fb_common(bool adjoint, const float* grad_w_hat, const float*
   p.ck64_stride = lay.ck64_stride;
   p.part_stride = lay.part_stride;
   p.row = lay.row;
-  p.sqsc = std::sqrt(1.4426950408889634 / static_cast<double>(T));
+  // the kernels carry every float64 log2-domain value times 2^128, the scaled weights and codewords times 2^64
+  p.sqsc = std::ldexp(std::sqrt(1.4426950408889634 / static_cast<double>(T)), 64);
   p.two_over_T = static_cast<float>(2.0 / static_cast<double>(T));
   p.L = L;
   p.k = k;

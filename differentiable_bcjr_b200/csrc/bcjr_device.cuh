@@ -223,22 +223,27 @@ constexpr long long kWaitLimitCycles = 4000000000LL;
 // Wait for the phase with the given parity to complete (acquire at cluster
 // scope, so the other CTAs' st.async data is visible).  Gives up after
 // `limit` SM clock cycles, ORs `timeout_bit` into *status and returns false.
+// One try: true once the phase with the given parity has completed.  The hint
+// lets the thread sleep in hardware until the phase completes (or 0.1 ms
+// pass) instead of re-issuing a loop.
+__device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(a), "r"(parity), "r"(100000u)
+      : "memory");
+  return done != 0;
+}
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, int timeout_bit,
                                           long long limit = kWaitLimitCycles) {
   const uint32_t a = smem_u32(bar);
-  uint32_t done = 0;
+  if (mbar_try(a, parity)) return true;  // the usual case: no clock reads
   const long long t0 = clock64();
   while (true) {
-    // The hint lets the thread sleep in hardware until the phase completes
-    // (or 0.1 ms pass) instead of re-issuing the loop.
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done)
-        : "r"(a), "r"(parity), "r"(100000u)
-        : "memory");
-    if (done) return true;
+    if (mbar_try(a, parity)) return true;
     if (clock64() - t0 > limit) {
       atomicOr(status, timeout_bit);
       return false;

@@ -37,9 +37,10 @@ struct FBParams {
   // thread tt of the team owns elements [tt*NV, tt*NV + NV) of every row, so a
   // row holds team_threads * NV values (= S/2^k for k <= 2, S/4 for k >= 3,
   // where lanes sharing a forward group each keep their own copy).
-  float* ck;               // C == 1: [n][row] forward values A'_t - R - 1 (float); C > 1: ring [C][row]
-  uint32_t* ckR;           // C == 1: [n][team_threads] high word of each thread's reference R; C > 1: ring [C][...]
-  float* ckF;              // same layout as ck for the forward adjoint accumulators (backward)
+  // Forward values A_t (every float64 log2-domain value carries a factor 2^128):
+  float* ck;               // C == 1: [n][row] A_t - R (float, unscaled); C > 1: ring [C][row]
+  uint32_t* ckR;           // [n][team_threads] high word of each thread's reference R - 1; C > 1: ring
+  float* ckF;              // backward: same layout as ck for the forward adjoint accumulators
   double* ck64;            // C > 1: [n/C + 1][row] A'_t at t = 0, C, 2C, ... (float64)
   float* ckF64;            // C > 1: [n/C + 1][row] forward adjoint accumulators at the same t
   float* part;             // [n][2][warps_per_team] per-warp partial sums
@@ -49,7 +50,7 @@ struct FBParams {
   size_t ck64_stride;      // elements per lane in ck64 / ckF64
   size_t part_stride;      // floats per lane in part
   size_t row;              // elements per checkpoint row (team_threads * NV)
-  double sqsc;             // sqrt(log2(e) / T): emission phi = -((w - c) sqsc)^2 in log2 units
+  double sqsc;             // sqrt(log2(e) / T) * 2^64: emission phi * 2^128 = -((w - c) sqsc)^2
   float two_over_T;
   int L, k, n, N, C;
   int num_slots;
@@ -84,8 +85,9 @@ __host__ __device__ inline FBSmem fb_smem_layout(int GL, int NT, int NV, int nse
   l.per_team = static_cast<uint32_t>(nseq) * o;
   l.red = static_cast<uint32_t>(teams_per_cta) * l.per_team;
   o = l.red + 4u * 128u * 4u;
-  // staging of the stored forward values (C == 1 only; C > 1 reads its ring directly)
-  const uint32_t stg = alias ? static_cast<uint32_t>(nseq) * 2u * NT : 0u;
+  // staging of the stored forward values (C == 1 only; C > 1 reads its ring
+  // directly): NV floats, one reference word and (adjoint) NV accumulators
+  const uint32_t stg = alias ? static_cast<uint32_t>(nseq) * NT : 0u;  // one slot per sequence in flight
   l.stage = o;
   o += stg * NV * 4u;
   l.stageF = o;

@@ -193,10 +193,17 @@ cudaError_t fb_geometry_uncached(int L, int k, int n_seq, bool adjoint, int C, i
   const int NV = states_per_thread_values(k);
   const bool alias = (C == 1);
   const int max_smem = max_optin_smem();
-  (void)nseq_request;
-  // Clusters keep two sequences in flight (the barrier of one hides behind the
-  // other's step); k = 1 has twice the group values and keeps one.
-  const int nseq = (g->cluster > 1 && k >= 2) ? 2 : 1;
+  // Clusters keep several sequences in flight, so that the exchange wait and
+  // the barrier of one sequence's step hide behind the others' steps: two by
+  // default (measured fastest for both calls), or 3 or 4 on request for the
+  // soft-codeword call when they fit in shared memory; k = 1 has twice the
+  // group values and keeps one.
+  int nseq = (g->cluster > 1 && k >= 2) ? 2 : 1;
+  if (nseq_request != 0 && nseq == 2) {  // single-CTA and k = 1 teams ignore the request
+    if (nseq_request < 2 || nseq_request > 4 || (adjoint && nseq_request != 2))
+      return cudaErrorNotSupported;
+    nseq = nseq_request;
+  }
   const size_t smem = fb_smem_layout(GL, g->block_threads, NV, nseq, adjoint, alias, g->teams_per_cta).total;
   if (smem > static_cast<size_t>(max_smem)) return cudaErrorNotSupported;
   g->nseq = nseq;
@@ -212,7 +219,7 @@ cudaError_t fb_geometry(int L, int k, int n_seq, bool adjoint, int C, int nseq_r
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  const GeoKey key{dev, L, k, n_seq, adjoint ? 1 : 0, C == 1 ? 1 : 0, nseq_request == 1 ? 3 : 0};
+  const GeoKey key{dev, L, k, n_seq, adjoint ? 1 : 0, C == 1 ? 1 : 0, nseq_request};
   {
     std::lock_guard<std::mutex> lk(g_geo_mu);
     auto it = g_geo_cache.find(key);

@@ -77,7 +77,7 @@ class ShardedSoftQuant:
 
     def __init__(self, codebook: torch.Tensor, state_bits: int, k: int, group=None,
                  forward_fn: Optional[Forward] = None, backward_fn: Optional[Backward] = None,
-                 checkpoint_interval: int = 0):
+                 checkpoint_interval: int = 0, sequences_in_flight: int = 0):
         if forward_fn is None or backward_fn is None:
             from . import bcjr_backward, bcjr_forward
             forward_fn = forward_fn or bcjr_forward
@@ -87,13 +87,14 @@ class ShardedSoftQuant:
         self.k = int(k)
         self.group = group
         self.C = int(checkpoint_interval)
+        self.fwd_kw = {"sequences_in_flight": int(sequences_in_flight)} if sequences_in_flight else {}
         self._fwd = forward_fn
         self._bwd = backward_fn
         self._grad_c = None
 
     def forward(self, w_local: torch.Tensor, T: float, out: Optional[torch.Tensor] = None) -> torch.Tensor:
         w_hat, _, _ = self._fwd(w_local, self.codebook, T, self.state_bits, self.k,
-                                checkpoint_interval=self.C, out=out)
+                                checkpoint_interval=self.C, out=out, **self.fwd_kw)
         return w_hat
 
     def backward(self, g_local: torch.Tensor, w_local: torch.Tensor, w_hat_local: torch.Tensor,

@@ -59,9 +59,13 @@ typedef struct {
   /* Keep the forward group vector every C steps and recompute the others
    * during the backward sweep; 0 selects C = 1 (keep every step). */
   int checkpoint_interval;
-  /* Sequences a team keeps in flight; must be 0 (automatic: two per
-   * thread-block cluster when k >= 2, so that one sequence's step hides the
-   * other's barrier, and one otherwise).  Other values are rejected. */
+  /* Sequences a thread-block-cluster team (state_bits >= 14) keeps in
+   * flight, so that one sequence's exchange and barrier hide behind the
+   * others' steps.  0 = automatic (two when k >= 2, one for k = 1).  2, 3 or 4
+   * may be requested for bcjr_forward with k >= 2 (BCJR_ERR_UNSUPPORTED when
+   * the buffers do not fit in shared memory), 2 for bcjr_backward; values
+   * outside 0..4 are BCJR_ERR_INVALID_ARG.  Ignored by single-CTA teams; the
+   * dense calls accept only 0. */
   int sequences_in_flight;
   /* Testing aid for the bounded device-side waits; 0 in normal use.  When
    * positive, a bcjr_forward / bcjr_backward call whose team is a

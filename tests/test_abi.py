@@ -107,6 +107,26 @@ class _Opts(ctypes.Structure):
                 ("reserved", ctypes.c_int * 6)]
 
 
+class _BitshiftOpts(ctypes.Structure):
+    _fields_ = [("checkpoint_interval", ctypes.c_int), ("sequences_in_flight", ctypes.c_int),
+                ("timeout_probe_cycles", ctypes.c_int), ("reserved", ctypes.c_int * 5)]
+
+
+def test_bitshift_options_are_checked_on_the_host(lib):
+    INVALID = 1
+    f = lib.bcjr_forward
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                  ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(_BitshiftOpts),
+                  ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    for field, value in [("sequences_in_flight", 5), ("sequences_in_flight", -1), ("checkpoint_interval", -2),
+                         ("timeout_probe_cycles", -1)]:
+        o = _BitshiftOpts()
+        setattr(o, field, value)
+        # fake, never-dereferenced addresses: rejected before any CUDA call
+        assert f(4096, 8192, 0.5, 16, 2, 8, 2, 12288, None, None, ctypes.pointer(o), 65536, 1 << 30, None) == INVALID
+
+
 def test_dense_arguments_are_rejected_on_the_host(lib):
     INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 3
     f = lib.bcjr_dense_forward

@@ -88,6 +88,20 @@ def test_cluster_team_marginals(B, L, k, n, N, T):
     np.testing.assert_allclose(to_np(log_z), o_lz, rtol=LOGZ_RTOL, atol=1e-4)
 
 
+@pytest.mark.parametrize("L,k,nseq", [(16, 2, 2), (16, 2, 3), (16, 2, 4), (15, 3, 3), (14, 4, 4)])
+def test_sequences_in_flight(B, L, k, nseq):
+    # the forward call with 2, 3 or 4 sequences in flight per cluster team, on a
+    # batch that leaves the last round of teams partly idle
+    n, N, T = 9, 7, 0.2
+    c, w, _ = _case(L, k, n, N, seed=700 + nseq)
+    w_hat, marg, log_z = B.bcjr_forward(w.cuda(), c.cuda(), T, L, k, want_marginals=True,
+                                        sequences_in_flight=nseq)
+    o_what, o_lz, o_gamma = oracle.forward(w, c, T, L, k, want_gamma=True)
+    assert_abs(w_hat, o_what, W_HAT_ATOL, f"w_hat nseq={nseq}")
+    assert_abs(marg, o_gamma, MARGINAL_ATOL, f"marginals nseq={nseq}")
+    np.testing.assert_allclose(to_np(log_z), o_lz, rtol=LOGZ_RTOL, atol=1e-4)
+
+
 @pytest.mark.parametrize("L,k,n,N,T,C", [(8, 2, 13, 3, 0.5, 4), (10, 3, 12, 2, 0.3, 3),
                                            (16, 2, 11, 2, 0.2, 4), (12, 2, 9, 2, 0.4, 9),
                                            (9, 1, 10, 2, 0.6, 2), (15, 4, 7, 2, 0.3, 5)])
