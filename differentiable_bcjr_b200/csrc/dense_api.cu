@@ -49,6 +49,42 @@ DenseLayout dense_layout(int grid, int n, bool adjoint, int dl_parts = 0) {
   return l;
 }
 
+// Workspace of the forward call (tensor cores): the transfer matrix as two
+// sets of resident operand slices, the emission reference of every step, and
+// per CTA of the resident clusters its forward vectors and partial sums.
+struct DenseTCLayout {
+  size_t Bfwd, Bbwd, mtab, ck, part, total, ck_stride, part_stride;
+};
+
+DenseTCLayout dense_tc_layout(int clusters, int n, int N) {
+  const size_t S = bcjr::kDenseStates, R = bcjr::kDenseTCRows, CL = bcjr::kDenseTCCluster;
+  DenseTCLayout l = {};
+  l.ck_stride = static_cast<size_t>(n) * R * (S / CL);
+  l.part_stride = static_cast<size_t>(2 * n + 1) * R * 2;
+  const size_t ctas = static_cast<size_t>(clusters) * CL;
+  size_t off = kHeader;
+  l.Bfwd = off;
+  off = align_up(off + S * S * 2 * sizeof(float));
+  l.Bbwd = off;
+  off = align_up(off + S * S * 2 * sizeof(float));
+  l.mtab = off;
+  off = align_up(off + static_cast<size_t>(N) * n * sizeof(float));
+  l.ck = off;
+  off = align_up(off + ctas * l.ck_stride * sizeof(float));
+  l.part = off;
+  off = align_up(off + ctas * l.part_stride * sizeof(float));
+  l.total = off;
+  return l;
+}
+
+bcjr_status dense_tc_clusters(int N, int* clusters) {
+  const int cap = bcjr::dense_tc_max_clusters();
+  if (cap < 1) return BCJR_ERR_UNSUPPORTED;
+  const int tiles = (N + bcjr::kDenseTCRows - 1) / bcjr::kDenseTCRows;
+  *clusters = tiles < 1 ? 1 : (tiles < cap ? tiles : cap);
+  return BCJR_OK;
+}
+
 // Launch geometry of the backward call that also returns the log-transition
 // gradient: the rows of that gradient live in per-CTA regions, so every CTA
 // takes one block of 32 sequences per launch and longer batches run in chunks
@@ -108,6 +144,33 @@ bcjr_status dense_common(bool adjoint, const float* g, const float* w, const flo
     if (marginals && !aligned(marginals, 16)) return BCJR_ERR_INVALID_ARG;
   }
   if (!ws || !aligned(ws, kAlign)) return BCJR_ERR_WORKSPACE;
+  if (!adjoint) {
+    // The soft codeword: the tensor-core kernel (dense_tc_kernel.cu).
+    int clusters = 0;
+    if ((st = dense_tc_clusters(N, &clusters)) != BCJR_OK) return st;
+    const DenseTCLayout lt = dense_tc_layout(clusters, n, N);
+    if (ws_bytes < lt.total) return BCJR_ERR_WORKSPACE;
+    char* b = static_cast<char*>(ws);
+    bcjr::DenseTCParams tp = {};
+    tp.w = w;
+    tp.codebook = c;
+    tp.mtab = reinterpret_cast<float*>(b + lt.mtab);
+    tp.Bfwd = reinterpret_cast<float*>(b + lt.Bfwd);
+    tp.Bbwd = reinterpret_cast<float*>(b + lt.Bbwd);
+    tp.ck = reinterpret_cast<float*>(b + lt.ck);
+    tp.part = reinterpret_cast<float*>(b + lt.part);
+    tp.w_hat = w_hat;
+    tp.marginals = marginals;
+    tp.log_z = log_z;
+    tp.status = reinterpret_cast<int*>(b);
+    tp.ck_stride = lt.ck_stride;
+    tp.part_stride = lt.part_stride;
+    tp.sc2 = static_cast<float>(1.4426950408889634 / static_cast<double>(T));
+    tp.n = n;
+    tp.N = N;
+    if ((st = from_cuda(cudaMemsetAsync(ws, 0, sizeof(int), s))) != BCJR_OK) return st;
+    return from_cuda(bcjr::launch_dense_tc_forward(tp, lam, clusters, s));
+  }
   const bool dl = adjoint && grad_lam;
   int grid = 0, chunk = N, parts = 0;
   if (dl) {
@@ -200,6 +263,11 @@ size_t bcjr_dense_workspace_size_impl(int op, int n_states, int seq_len, int n_s
     int chunk = 0, parts = 0;
     if (dlam_geometry(n_seq > 0 ? n_seq : 1, &grid, &chunk, &parts) != BCJR_OK) return 0;
     return dense_layout(grid, seq_len, true, parts).total;
+  }
+  if (!adjoint) {
+    int clusters = 0;
+    if (dense_tc_clusters(n_seq > 0 ? n_seq : 1, &clusters) != BCJR_OK) return 0;
+    return dense_tc_layout(clusters, seq_len, n_seq > 0 ? n_seq : 1).total;
   }
   if (bcjr::dense_geometry(adjoint, n_seq > 0 ? n_seq : 1, &grid) != cudaSuccess) return 0;
   return dense_layout(grid, seq_len, adjoint).total;

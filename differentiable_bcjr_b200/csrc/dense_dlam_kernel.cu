@@ -36,9 +36,11 @@
 
 #include "bcjr_device.cuh"
 #include "dense_internal.h"
+#include "tc_util.cuh"
 
 namespace bcjr {
 namespace dlam {
+using namespace tc;
 
 constexpr int kS = kDenseStates;                    // 256
 constexpr int kK = 8;                               // rows per stage (one tf32 MMA step)
@@ -48,65 +50,6 @@ constexpr int kTiles = 8;                           // X hi/lo, U hi/lo, W hi/lo
 constexpr uint32_t kStageBytes = kTiles * kTileBytes;  // 64 KiB
 constexpr int kStages = 2;
 constexpr uint32_t kTmemCols = 512;                 // 2 x (M = 128 lanes, N = 256 columns) float32
-
-// Byte offset of the 16-byte chunk (row m, K-chunk kc) in a K-major core-matrix
-// tile: a core matrix is 8 rows x 16 bytes stored contiguously; the two K
-// chunks of a row group are 128 bytes apart (leading byte offset) and row
-// groups 256 bytes apart (stride byte offset).
-__device__ __forceinline__ uint32_t chunk_off(int m, int kc) {
-  return static_cast<uint32_t>(((m >> 3) * 2 + kc) * 128 + (m & 7) * 16);
-}
-// Shared-memory matrix descriptor of such a tile starting at `saddr`:
-// start address, leading byte offset 128, stride byte offset 256 (all >> 4),
-// descriptor version 1, no swizzle.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr) {
-  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(128u >> 4) << 16) |
-         (static_cast<uint64_t>(256u >> 4) << 32) | (1ull << 46);
-}
-// Instruction descriptor: float32 accumulator, tf32 A and B, both K-major,
-// N = 256, M = 128.
-constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((256u >> 3) << 17) | ((128u >> 4) << 24);
-
-__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate), "r"(0u)
-      : "memory");
-}
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void async_proxy_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
-// x = hi + lo with hi = x rounded to tf32 (low 13 mantissa bits zero) and
-// lo = x - hi, exact in float32.
-__device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
-  uint32_t h;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(x));
-  hi = __uint_as_float(h);
-  lo = x - hi;
-}
-
-// 32 consecutive float32 columns of this warp's 32 TMEM lanes.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
 
 }  // namespace dlam
 

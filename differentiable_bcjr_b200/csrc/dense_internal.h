@@ -38,6 +38,31 @@ struct DenseParams {
   int n, N;
 };
 
+// Soft codeword of the dense trellis on the tensor cores (dense_tc_kernel.cu):
+// a cluster of kDenseTCCluster CTAs per kDenseTCRows sequences, CTA r holding
+// K-slice r of the transfer matrix.
+constexpr int kDenseTCCluster = 4;
+constexpr int kDenseTCRows = 128;
+
+struct DenseTCParams {
+  const float* w;          // [N][n]
+  const float* codebook;   // [S]
+  float* mtab;             // [N][n] emission reference of every step (written by the reference kernel)
+  float* Bfwd;             // [4 slices][128 KiB] P as resident operand tiles (forward sweep)
+  float* Bbwd;             // the same for P^T (backward sweep)
+  float* ck;               // per CTA [n][16][128] float4: forward vectors, this CTA's 64 states
+  float* part;             // per CTA [n][2 halves][128][2] partial sums (sum c gamma, sum gamma) over
+                           // 32 states each, then [128][2 halves] the last forward vector's row sums
+  float* w_hat;            // [N][n]
+  float* marginals;        // [N][n][S] or null
+  float* log_z;            // [N] or null
+  int* status;
+  size_t ck_stride;        // floats per CTA in ck
+  size_t part_stride;      // floats per CTA in part
+  float sc2;               // log2(e) / T
+  int n, N;
+};
+
 // Log-transition gradient of the dense trellis (dense_dlam_kernel.cu): rows of
 // X, U, V, W written by the backward kernel, one region per backward CTA
 // (`region_stride` floats apart), `spr` stages of 8 rows per region.
@@ -60,6 +85,9 @@ int dense_max_grid(bool adjoint);
 cudaError_t launch_dense_prep(const float* lam, const DenseParams& p, cudaStream_t s);
 cudaError_t launch_dense(const DenseParams& p, const float* lam, bool adjoint, int grid, cudaStream_t s,
                          bool prep = true);
+size_t dense_tc_smem_bytes();
+int dense_tc_max_clusters();
+cudaError_t launch_dense_tc_forward(const DenseTCParams& p, const float* lam, int clusters, cudaStream_t s);
 size_t dlam_smem_bytes();
 cudaError_t dlam_grid(long long total_stages, int* grid);
 cudaError_t launch_dlam(const DlamParams& p, int grid, cudaStream_t s);

@@ -1,0 +1,553 @@
+// dense_tc_kernel.cu -- soft codeword of the dense (fully connected) trellis on
+// the fifth-generation tensor cores (tcgen05, sm_100a).
+//
+// "BCJR-QAT: A Differentiable Relaxation of Trellis-Coded Weight Quantization",
+// abstract: the relaxation is a 1D Ising-like chain solved by a transfer
+// matrix.  With P = exp(Lambda) (row = source state) and emission factors
+// E_t(s) = 2^(phi_t(s) - m_t), phi_t(s) = -(w_t - c(s))^2 log2(e) / T and m_t the
+// largest phi_t of the step, the probability-domain recursions are
+//   forward   u_0 = E_0,            u_t = ((u_{t-1} P) (.) E_t) / s_{t-1},
+//   backward  z_{n-1} = 1,          z_{t-1} = ((E_t (.) z_t) P^T) / sigma_t,
+//   gamma_t = u_t (.) z_t / sum_s u_t(s) z_t(s),   w_hat_t = sum_s c(s) gamma_t(s),
+// with s_t = sum_s u_t(s) and sigma_t = sum_s E_t(s) z_t(s): any per-row scale
+// cancels in gamma, and dividing by the previous step's sum keeps every row's
+// sum in (0, 1] (P is row-stochastic for the normalised Lambda, and within a
+// step's column-sum spread in general).  log2 Z = sum_t m_t + sum_t log2 s_t.
+//
+// Each step is one [rows x 256] x [256 x 256] contraction: a real batched
+// matrix product, run here as three tf32 products (x = hi + lo, hi*hi + hi*lo +
+// lo*hi: float32-level accuracy; one tf32 product would leave ~5e-4 relative
+// error in a step's dominant terms).
+//
+// Work split.  A thread-block cluster of 4 CTAs owns 128 sequences (the MMA's
+// M = 128).  CTA r keeps K-slice r of the transfer matrix (input states
+// 64r .. 64r+63, as tf32 head and tail in K-major core-matrix tiles, 128 KiB)
+// resident in shared memory; its operand A, the same 64 states of the current
+// vector as head and tail, lives in tensor memory next to the accumulator.
+// The 96 MMAs of a step (4 output blocks of 64 states x 8 K-chunks x 3
+// products) give partial sums for all 256 output states; CTA r's output states
+// 64r .. 64r+63 are exactly its next K-slice, so only the partial sums cross
+// CTAs (a reduce-scatter over distributed shared memory) and the operand never
+// does.  The output blocks are issued and committed one at a time, the other
+// CTAs' blocks first, so sending a finished block (st.async from the sending
+// warps' registers, completing on the receiver's mbarrier) overlaps the MMAs
+// of the next.  Four warps own the CTA's 64 output states of one row each:
+// they add the three received blocks to their own, scale and store the new
+// vector, and write it back to tensor memory as the next operand.  Each row's
+// sum over the CTA's states rides along with the next step's blocks (for the
+// next normalisation).  A split cluster barrier per step keeps a CTA from
+// overwriting a receive buffer that another CTA is still reading.  The
+// backward sweep reloads the resident slice with P's other orientation.  The
+// per-step reference m_t comes from a small kernel that finds each weight's
+// nearest codeword.
+#include <cuda_runtime.h>
+
+#include <cfloat>
+#include <cmath>
+#include <cstdint>
+
+#include "bcjr_device.cuh"
+#include "dense_internal.h"
+#include "tc_util.cuh"
+
+namespace bcjr {
+namespace dtc {
+
+using namespace tc;
+
+constexpr int kS = kDenseStates;            // 256 states
+constexpr int kCL = kDenseTCCluster;        // 4 CTAs per cluster = K-slices
+constexpr int kSlice = kS / kCL;            // 64 states per CTA
+constexpr int kKC = kSlice / 8;             // 8 K-chunks of 8 states
+constexpr int kMR = kDenseTCRows;           // 128 sequences per cluster tile (MMA M)
+constexpr int kThreads = 256;
+constexpr int kGroups = kSlice / 4;         // 16 groups of 4 states in a row's block
+constexpr uint32_t kBTile = kS * 8 * 4;     // [256 rows][8 k] tf32 tile: 8 KiB
+constexpr uint32_t kBBytes = kKC * 2 * kBTile;        // 8 K-chunks x (head, tail): 128 KiB
+constexpr uint32_t kBBlock = 64 / 8 * 256;            // byte offset of the next 64 output rows in a tile
+constexpr uint32_t kRxData = kMR * kSlice * 4;        // one sender's block: [16 groups][128 rows] float4, 32 KiB
+constexpr uint32_t kRxSlot = kRxData + kMR * 4;       // + the sender's row sums [128]
+constexpr uint32_t kRxBytes = (kCL - 1) * kRxSlot;    // bytes received per exchange
+constexpr uint32_t kOnesBytes = 16 * 8 * 4;        // [16 rows][8 k] tile of ones: row sums on the tensor cores
+constexpr uint32_t kOffB = 0, kOffRx = kBBytes, kOffOnes = kOffRx + kRxBytes;
+constexpr uint32_t kOffBar = kOffOnes + kOnesBytes;
+constexpr uint32_t kSmemBytes = kOffBar + 64;
+static_assert(kSmemBytes <= 227u * 1024u, "shared memory");
+// Tensor memory: accumulator in columns [0, 256), operand head [256, 320) and
+// tail [320, 384), the operand's row sums over this CTA's states in [384, 400).
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTAh = kS, kTAl = kS + kSlice, kTSum = kS + 2 * kSlice;
+constexpr uint32_t kIdescN64 = idesc_tf32(64), kIdescN16 = idesc_tf32(16);
+
+__device__ __forceinline__ void st_async_v4f32(uint32_t raddr, float a, float b, float c, float d, uint32_t rbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   raddr),
+               "f"(a), "f"(b), "f"(c), "f"(d), "r"(rbar)
+               : "memory");
+}
+// Bulk copy global -> this CTA's shared memory, completing `bytes` on `bar`.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+}  // namespace dtc
+
+// The transfer matrix as resident slices: slice r of the forward image holds,
+// for output state n and input state k in [64r, 64r+64), P[k][n]; slice r of
+// the backward image holds P[n][k] (the product with P^T).  Each slice is
+// [K-chunk c][head, tail][256 rows n][8 k] in K-major core-matrix tiles.
+__global__ void dense_tc_prep_kernel(const float* __restrict__ lam, float* __restrict__ Bfwd,
+                                     float* __restrict__ Bbwd) {
+  using namespace dtc;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= kS * kS) return;
+  const int row = i / kS, col = i - row * kS;
+  float hi, lo;
+  split_tf32(expf(lam[i]), hi, lo);  // P[row][col]
+  auto put = [&](float* B, int nn, int kk) {
+    const int r = kk / kSlice, c = (kk % kSlice) / 8, kc = (kk & 7) >> 2, e = kk & 3;
+    unsigned char* base = reinterpret_cast<unsigned char*>(B) + static_cast<size_t>(r) * kBBytes + c * 2 * kBTile;
+    const uint32_t off = chunk_off(nn, kc) + 4u * e;
+    *reinterpret_cast<float*>(base + off) = hi;
+    *reinterpret_cast<float*>(base + kBTile + off) = lo;
+  };
+  put(Bfwd, col, row);  // forward: output state col, input state row
+  put(Bbwd, row, col);  // backward: output state row, input state col
+}
+
+// Reference of every (sequence, step): m = max_s -(w - c(s))^2 log2(e)/T, the
+// value at the codeword nearest to w, computed with the same float operations
+// as the emissions so that every factor 2^(phi - m) is at most one.
+__global__ void dense_tc_mtab_kernel(const float* __restrict__ w, const float* __restrict__ codebook, float sc2,
+                                     long long total, float* __restrict__ mtab) {
+  using namespace dtc;
+  __shared__ float cs[kS];
+  const int tid = threadIdx.x;  // blockDim.x == kS
+  const float ci = codebook[tid];
+  int rank = 0;
+  for (int j = 0; j < kS; ++j) {
+    const float cj = codebook[j];
+    rank += (cj < ci) || (cj == ci && j < tid);
+  }
+  cs[rank & (kS - 1)] = ci;
+  __syncthreads();
+  for (long long i = static_cast<long long>(blockIdx.x) * kS + tid; i < total; i += static_cast<long long>(gridDim.x) * kS) {
+    const float wv = w[i];
+    int lo = 0, hi = kS;  // first index with cs[idx] >= wv
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (cs[mid] < wv) {
+        lo = mid + 1;
+      } else {
+        hi = mid;
+      }
+    }
+    float best = -FLT_MAX;
+    if (lo < kS) {
+      const float d = wv - cs[lo];
+      best = fmaxf(best, -(d * d) * sc2);
+    }
+    if (lo > 0) {
+      const float d = wv - cs[lo - 1];
+      best = fmaxf(best, -(d * d) * sc2);
+    }
+    mtab[i] = best;
+  }
+}
+
+__global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::kThreads, 1)
+    dense_tc_fwd_kernel(const DenseTCParams p) {
+  using namespace dtc;
+  extern __shared__ __align__(16) unsigned char sm[];
+  unsigned char* Bs = sm + kOffB;
+  unsigned char* Rx = sm + kOffRx;
+  float* ones = reinterpret_cast<float*>(sm + kOffOnes);
+  uint64_t* bar_c = reinterpret_cast<uint64_t*>(sm + kOffBar);  // [4] output blocks committed, in issue order
+  uint64_t* bar_rx = bar_c + 4;                                  // the three blocks of an exchange received
+  uint64_t* bar_b = bar_c + 5;                                   // resident slice loaded
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_c + 6);
+  int* abort_flag = reinterpret_cast<int*>(bar_c + 7);
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int r = static_cast<int>(cluster_rank());
+  const int cid = static_cast<int>(blockIdx.x) / kCL, ncl = static_cast<int>(gridDim.x) / kCL;
+  // Thread (half, row): states 32 half .. 32 half + 31 of every 64-state block
+  // of row `row`, which is tensor-memory lane `row`.
+  const int half = warp >> 2;
+  const int row = (warp & 3) * 32 + (tid & 31);
+  const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  const int n = p.n, N = p.N;
+  const int ntiles = (N + kMR - 1) / kMR;
+  const float sc2 = p.sc2;
+
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (tid == 0) {
+    for (int i = 0; i < 6; ++i) mbar_init(bar_c + i, 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (tid < kOnesBytes / 4) ones[tid] = 1.f;
+  async_proxy_fence();  // the ones tile is read by the tensor cores
+  float cw[32];         // codewords of this thread's states
+#pragma unroll
+  for (int j = 0; j < 32; ++j) cw[j] = __ldg(p.codebook + r * kSlice + 32 * half + j);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (tid == 0) mbar_arm(bar_rx, kRxBytes);
+  cluster_sync_all();  // every CTA's barriers are initialised (and armed) before any remote store
+
+  uint32_t ph_c[4] = {0, 0, 0, 0}, ph_rx = 0, ph_b = 0;
+  // After one wait of this CTA gave up, no thread waits again (the call's results are void).
+  auto waitb = [&](uint64_t* bar, uint32_t& ph) {
+    if (!*reinterpret_cast<volatile int*>(abort_flag) && !mbar_wait(bar, ph, p.status, kDevTimeout))
+      *reinterpret_cast<volatile int*>(abort_flag) = 1;
+    ph ^= 1u;
+  };
+
+  // Load a resident slice (tid 0), completing on bar_b.
+  auto load_b = [&](const float* image) {
+    if (tid == 0) {
+      mbar_arm(bar_b, kBBytes);
+      const unsigned char* src = reinterpret_cast<const unsigned char*>(image) + static_cast<size_t>(r) * kBBytes;
+#pragma unroll 1
+      for (int q = 0; q < 8; ++q)
+        bulk_g2s(smem_u32(Bs) + q * (kBBytes / 8), src + q * (kBBytes / 8), kBBytes / 8, smem_u32(bar_b));
+    }
+  };
+  // Output block of issue slot k: the other CTAs' blocks first, the own one last.
+  auto block_of = [&](int k) { return (r + 1 + k) & (kCL - 1); };
+  // The MMAs of one step (tid 0), one commit per output block; the operand's
+  // row sums over this CTA's states (head and tail times a tile of ones) go
+  // with the first block.
+  auto issue_mma = [&](bool first_of_sweep) {
+    if (first_of_sweep) waitb(bar_b, ph_b);
+    tc_fence_after();
+    const bool go = !*reinterpret_cast<volatile int*>(abort_flag);
+    const uint32_t b0 = smem_u32(Bs);
+#pragma unroll 1
+    for (int k = 0; k < kCL; ++k) {
+      const int blk = block_of(k);
+      const uint32_t d = tmem + static_cast<uint32_t>(blk * kSlice);
+      if (go) {
+        if (k == 0) {
+          const uint64_t od = smem_desc(smem_u32(ones));
+#pragma unroll
+          for (int c = 0; c < kKC; ++c) {
+            mma_tf32_ts(tmem + kTSum, tmem + kTAh + 8 * c, od, kIdescN16, c > 0 ? 1u : 0u);
+            mma_tf32_ts(tmem + kTSum, tmem + kTAl + 8 * c, od, kIdescN16, 1u);
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < kKC; ++c) {
+          const uint32_t bh = b0 + (2 * c) * kBTile + blk * kBBlock, bl = bh + kBTile;
+          const uint32_t ah = tmem + kTAh + 8 * c, al = tmem + kTAl + 8 * c;
+          mma_tf32_ts(d, ah, smem_desc(bh), kIdescN64, c > 0 ? 1u : 0u);  // hi * hi
+          mma_tf32_ts(d, ah, smem_desc(bl), kIdescN64, 1u);               // hi * lo
+          mma_tf32_ts(d, al, smem_desc(bh), kIdescN64, 1u);               // lo * hi
+        }
+      }
+      mma_commit(bar_c + k);
+    }
+  };
+  // One step's contraction and reduce-scatter.  Every thread sends its half of
+  // the other CTAs' blocks of its row as they complete (st.async into the
+  // receiver's slot: 16 groups x 128 rows of float4, so a warp's stores are
+  // contiguous; half 0 adds the row sum), then adds the three received halves
+  // to its own into y.  Returns the row's sum of the consumed vector over all
+  // 256 states, added in CTA order so that every CTA gets the same value.
+  auto step = [&](bool first_of_sweep, float (&y)[32]) -> float {
+    tc_fence_before();
+    __syncthreads();  // operand written, accumulator read: the MMAs may go
+    if (tid == 0) issue_mma(first_of_sweep);
+    __syncwarp();
+    cluster_wait_plain();  // every CTA has read its receive buffer of the previous exchange
+    float rs = 0.f;        // this CTA's part of the row sum
+#pragma unroll 1
+    for (int k = 0; k < kCL - 1; ++k) {
+      const int blk = block_of(k);
+      waitb(bar_c + k, ph_c[k]);
+      tc_fence_after();
+      uint32_t v[32];
+      tmem_ld32_async(tmem + lane_off + static_cast<uint32_t>(blk * kSlice + 32 * half), v);
+      if (k == 0) {
+        uint32_t s1;
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(s1) : "r"(tmem + lane_off + kTSum));
+        tmem_wait_ld();
+        rs = __uint_as_float(s1);
+      } else {
+        tmem_wait_ld();
+      }
+      const uint32_t slot = static_cast<uint32_t>(r < blk ? r : r - 1);
+      const uint32_t dst = mapa_u32(smem_u32(Rx) + slot * kRxSlot, static_cast<uint32_t>(blk));
+      const uint32_t rbar = mapa_u32(smem_u32(bar_rx), static_cast<uint32_t>(blk));
+#pragma unroll
+      for (int g = 0; g < 8; ++g)
+        st_async_v4f32(dst + static_cast<uint32_t>(((8 * half + g) * kMR + row) * 16), __uint_as_float(v[4 * g]),
+                       __uint_as_float(v[4 * g + 1]), __uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3]),
+                       rbar);
+      if (half == 0) st_async_f32(dst + kRxData + static_cast<uint32_t>(row * 4), rs, rbar);
+    }
+    waitb(bar_c + kCL - 1, ph_c[kCL - 1]);  // the last commit: every MMA of the step is done
+    tc_fence_after();
+    {
+      uint32_t v[32];
+      tmem_ld32_async(tmem + lane_off + static_cast<uint32_t>(r * kSlice + 32 * half), v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) y[j] = __uint_as_float(v[j]);
+    }
+    tc_fence_before();
+    waitb(bar_rx, ph_rx);
+    if (tid == 0) mbar_arm(bar_rx, kRxBytes);  // the next exchange's phase
+    float s = 0.f;
+#pragma unroll 1
+    for (int src = 0; src < kCL; ++src) {
+      if (src == r) {
+        s += rs;
+        continue;
+      }
+      const unsigned char* slot = Rx + (src < r ? src : src - 1) * kRxSlot;
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        const float4 q4 = *reinterpret_cast<const float4*>(slot + ((8 * half + g) * kMR + row) * 16);
+        y[4 * g] += q4.x;
+        y[4 * g + 1] += q4.y;
+        y[4 * g + 2] += q4.z;
+        y[4 * g + 3] += q4.w;
+      }
+      s += *reinterpret_cast<const float*>(slot + kRxData + row * 4);
+    }
+    cluster_arrive_relaxed();  // this CTA's receive buffer is read
+    return s;
+  };
+  // The next MMA's operand A: this thread's 32 values as tf32 head and tail.
+  auto put_operand = [&](const float (&v)[32]) {
+    uint32_t h[32], l[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      float fh, fl;
+      split_tf32(v[j], fh, fl);
+      h[j] = __float_as_uint(fh);
+      l[j] = __float_as_uint(fl);
+    }
+    tmem_st32(tmem + lane_off + kTAh + 32 * half, h);
+    tmem_st32(tmem + lane_off + kTAl + 32 * half, l);
+    tmem_wait_st();
+  };
+
+  float* ckbase = p.ck + static_cast<size_t>(cid * kCL + r) * p.ck_stride;      // [t][16 groups][128 rows] float4
+  // [t][half][128 rows][2] partial sums, then [128 rows][half] the last forward row sums
+  float* ptbase = p.part + static_cast<size_t>(cid * kCL + r) * p.part_stride;
+  auto ck_at = [&](int t, int g) {
+    return ckbase + ((static_cast<size_t>(t) * kGroups + 8 * half + g) * kMR + row) * 4;
+  };
+
+  for (int tile = cid; tile < ntiles; tile += ncl) {
+    const int q = tile * kMR + row;
+    const bool act = q < N;
+    const size_t qb = static_cast<size_t>(act ? q : 0) * n;  // padding rows run sequence 0 (discarded)
+
+    // ---------------- forward sweep ----------------
+    if (n > 1) load_b(p.Bfwd);  // one step has no contraction
+    cluster_arrive_relaxed();   // pairs with the first step's wait
+    double lsc = 0.0;           // log2 Z of the row: the references and log2 of the row sums
+    float wn = __ldg(p.w + qb), mn = __ldg(p.mtab + qb);  // the step's weight and reference, loaded a step ahead
+    float ps = 0.f;                                       // this thread's part of the current vector's row sum
+    for (int t = 0; t < n; ++t) {
+      float y[32];
+      float sprev = 1.f;
+      if (t > 0) sprev = step(t == 1, y);
+      const float wt = wn, mt = mn;
+      if (t + 1 < n) {
+        wn = __ldg(p.w + qb + t + 1);
+        mn = __ldg(p.mtab + qb + t + 1);
+      }
+      const float inv = 1.f / sprev;
+      ps = 0.f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float d = wt - cw[j];
+        const float e = ex2f(-(d * d) * sc2 - mt);
+        y[j] = (t > 0 ? y[j] * inv : 1.f) * e;
+        ps += y[j];
+      }
+      lsc += static_cast<double>(mt) + (t > 0 ? static_cast<double>(log2f(sprev)) : 0.0);
+#pragma unroll
+      for (int g = 0; g < 8; ++g)
+        *reinterpret_cast<float4*>(ck_at(t, g)) = make_float4(y[4 * g], y[4 * g + 1], y[4 * g + 2], y[4 * g + 3]);
+      if (t + 1 < n) put_operand(y);
+    }
+    // For log Z: the last vector's row sum, by CTA and half, in the row after the partial sums.
+    ptbase[static_cast<size_t>(n) * 4 * kMR + row * 2 + half] = ps;
+    cluster_wait_plain();  // pairs with the last arrive
+    cluster_sync_all();    // every CTA is done with the forward sweep's exchanges
+
+    // ---------------- backward sweep ----------------
+    if (n > 1) load_b(p.Bbwd);
+    cluster_arrive_relaxed();
+    wn = __ldg(p.w + qb + n - 1);
+    mn = __ldg(p.mtab + qb + n - 1);
+    for (int t = n - 1; t >= 0; --t) {
+      float z[32];
+      float4 x4[8];  // the stored forward vector of the step, requested before the exchange
+#pragma unroll
+      for (int g = 0; g < 8; ++g) x4[g] = *reinterpret_cast<const float4*>(ck_at(t, g));
+      float sig = 1.f;
+      if (t < n - 1) sig = step(t == n - 2, z);
+      const float wt = wn, mt = mn;
+      if (t >= 1) {
+        wn = __ldg(p.w + qb + t - 1);
+        mn = __ldg(p.mtab + qb + t - 1);
+      }
+      const float inv = 1.f / sig;
+      float den = 0.f, num = 0.f;
+#pragma unroll
+      for (int g = 0; g < 8; ++g) {
+        const float xs[4] = {x4[g].x, x4[g].y, x4[g].z, x4[g].w};
+        float gm[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = 4 * g + e;
+          z[j] = t < n - 1 ? z[j] * inv : 1.f;
+          gm[e] = xs[e] * z[j];
+          den += gm[e];
+          num = fmaf(gm[e], cw[j], num);
+        }
+        if (p.marginals && act)
+          *reinterpret_cast<float4*>(p.marginals + (static_cast<size_t>(q) * n + t) * kS + r * kSlice + 32 * half + 4 * g) =
+              make_float4(gm[0], gm[1], gm[2], gm[3]);
+      }
+      // Partial sums over this thread's 32 states: (sum c gamma, sum gamma), by half.
+      *reinterpret_cast<float2*>(ptbase + ((static_cast<size_t>(t) * 2 + half) * kMR + row) * 2) = make_float2(num, den);
+      if (t >= 1) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float d = wt - cw[j];
+          z[j] = ex2f(-(d * d) * sc2 - mt) * z[j];
+        }
+        put_operand(z);
+      }
+    }
+    cluster_wait_plain();
+    cluster_sync_all();  // every CTA's partial sums (and marginal rows) are written
+
+    // log Z (CTA 0, half 0): the forward references and row sums, and the last row sum over all states.
+    if (r == 0 && half == 0 && act) {
+      float s = 0.f;
+#pragma unroll
+      for (int src = 0; src < kCL; ++src)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          s += __ldcg(p.part + static_cast<size_t>(cid * kCL + src) * p.part_stride + static_cast<size_t>(n) * 4 * kMR +
+                      row * 2 + h);
+      const float lz = static_cast<float>((lsc + static_cast<double>(log2f(s))) * 0.69314718055994530942);
+      if (!isfinite(lz)) atomicOr(p.status, kDevNonFinite);
+      if (p.log_z) p.log_z[q] = lz;
+    }
+    // Soft codeword: CTA r takes the steps t = r, r + 4, ...; the partial sums
+    // over the 8 state blocks are added in a fixed order.
+    for (int t = r + kCL * (tid >> 7); t < n; t += 2 * kCL) {
+      const int rr = tid & (kMR - 1);
+      const int qq = tile * kMR + rr;
+      if (qq >= N) continue;
+      float num = 0.f, den = 0.f;
+#pragma unroll
+      for (int src = 0; src < kCL; ++src)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          // other CTAs wrote these (at addresses earlier tiles also used): read through L2
+          const float2 v = __ldcg(reinterpret_cast<const float2*>(
+              p.part + static_cast<size_t>(cid * kCL + src) * p.part_stride + ((static_cast<size_t>(t) * 2 + h) * kMR + rr) * 2));
+          num += v.x;
+          den += v.y;
+        }
+      p.w_hat[static_cast<size_t>(qq) * n + t] = num / den;
+    }
+    // Marginals: this CTA's 64 states of every step, divided by the step's sum.
+    if (p.marginals) {
+      for (int t = tid >> 7; t < n; t += 2) {
+        const int rr = tid & (kMR - 1);
+        const int qq = tile * kMR + rr;
+        if (qq >= N) continue;
+        float den = 0.f;
+#pragma unroll
+        for (int src = 0; src < kCL; ++src)
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            den += __ldcg(p.part + static_cast<size_t>(cid * kCL + src) * p.part_stride +
+                          ((static_cast<size_t>(t) * 2 + h) * kMR + rr) * 2 + 1);
+        const float inv = 1.f / den;
+        float* mr = p.marginals + (static_cast<size_t>(qq) * n + t) * kS + r * kSlice;
+#pragma unroll 4
+        for (int j = 0; j < kSlice; j += 4) {
+          float4 m4 = *reinterpret_cast<float4*>(mr + j);
+          m4.x *= inv;
+          m4.y *= inv;
+          m4.z *= inv;
+          m4.w *= inv;
+          *reinterpret_cast<float4*>(mr + j) = m4;
+        }
+      }
+    }
+    cluster_sync_all();  // partial sums read before the next tile rewrites them
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+  cluster_sync_all();  // no CTA leaves while its shared memory may be addressed
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+// ---------------------------------------------------------------------------
+size_t dense_tc_smem_bytes() { return dtc::kSmemBytes; }
+
+int dense_tc_max_clusters() {
+  const size_t smem = dense_tc_smem_bytes();
+  if (cudaFuncSetAttribute(dense_tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
+    return 0;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(dtc::kCL * sms, 1, 1);
+  cfg.blockDim = dim3(dtc::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, dense_tc_fwd_kernel, &cfg) != cudaSuccess) return 0;
+  return clusters;
+}
+
+cudaError_t launch_dense_tc_forward(const DenseTCParams& p, const float* lam, int clusters, cudaStream_t s) {
+  using namespace dtc;
+  dense_tc_prep_kernel<<<(kS * kS + 255) / 256, 256, 0, s>>>(lam, p.Bfwd, p.Bbwd);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long long total = static_cast<long long>(p.N) * p.n;
+  const long long blocks = (total + kS - 1) / kS;
+  dense_tc_mtab_kernel<<<static_cast<unsigned>(blocks < 4096 ? blocks : 4096), kS, 0, s>>>(p.w, p.codebook, p.sc2, total,
+                                                                                         p.mtab);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const size_t smem = dense_tc_smem_bytes();
+  if ((e = cudaFuncSetAttribute(dense_tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(smem))) != cudaSuccess)
+    return e;
+  dense_tc_fwd_kernel<<<clusters * kCL, kThreads, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace bcjr
