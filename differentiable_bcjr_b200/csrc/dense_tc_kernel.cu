@@ -60,7 +60,8 @@ constexpr int kCL = kDenseTCCluster;        // 4 CTAs per cluster = K-slices
 constexpr int kSlice = kS / kCL;            // 64 states per CTA
 constexpr int kKC = kSlice / 8;             // 8 K-chunks of 8 states
 constexpr int kMR = kDenseTCRows;           // 128 sequences per cluster tile (MMA M)
-constexpr int kThreads = 256;
+constexpr int kWorkers = 256;              // 8 warps: two per tensor-memory lane quadrant
+constexpr int kThreads = kWorkers + 32;     // + one warp that issues the MMAs
 constexpr int kGroups = kSlice / 4;         // 16 groups of 4 states in a row's block
 constexpr uint32_t kBTile = kS * 8 * 4;     // [256 rows][8 k] tf32 tile: 8 KiB
 constexpr uint32_t kBBytes = kKC * 2 * kBTile;        // 8 K-chunks x (head, tail): 128 KiB
@@ -70,8 +71,9 @@ constexpr uint32_t kRxSlot = kRxData + kMR * 4;       // + the sender's row sums
 constexpr uint32_t kRxBytes = (kCL - 1) * kRxSlot;    // bytes received per exchange
 constexpr uint32_t kOnesBytes = 16 * 8 * 4;        // [16 rows][8 k] tile of ones: row sums on the tensor cores
 constexpr uint32_t kOffB = 0, kOffRx = kBBytes, kOffOnes = kOffRx + kRxBytes;
-constexpr uint32_t kOffBar = kOffOnes + kOnesBytes;
-constexpr uint32_t kSmemBytes = kOffBar + 64;
+constexpr uint32_t kOffCw = kOffOnes + kOnesBytes;   // this CTA's 64 codewords
+constexpr uint32_t kOffBar = kOffCw + kSlice * 4;
+constexpr uint32_t kSmemBytes = kOffBar + 96;
 static_assert(kSmemBytes <= 227u * 1024u, "shared memory");
 // Tensor memory: accumulator in columns [0, 256), operand head [256, 320) and
 // tail [320, 384), the operand's row sums over this CTA's states in [384, 400).
@@ -164,18 +166,21 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
   unsigned char* Bs = sm + kOffB;
   unsigned char* Rx = sm + kOffRx;
   float* ones = reinterpret_cast<float*>(sm + kOffOnes);
+  const float* cws = reinterpret_cast<const float*>(sm + kOffCw);
   uint64_t* bar_c = reinterpret_cast<uint64_t*>(sm + kOffBar);  // [4] output blocks committed, in issue order
-  uint64_t* bar_rx = bar_c + 4;                                  // the three blocks of an exchange received
-  uint64_t* bar_b = bar_c + 5;                                   // resident slice loaded
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_c + 6);
-  int* abort_flag = reinterpret_cast<int*>(bar_c + 7);
+  uint64_t* bar_rx = bar_c + 4;                                  // [3] a receive slot filled
+  uint64_t* bar_b = bar_c + 7;                                   // resident slice loaded
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_c + 8);
+  int* abort_flag = reinterpret_cast<int*>(bar_c + 9);
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int r = static_cast<int>(cluster_rank());
   const int cid = static_cast<int>(blockIdx.x) / kCL, ncl = static_cast<int>(gridDim.x) / kCL;
-  // Thread (half, row): states 32 half .. 32 half + 31 of every 64-state block
-  // of row `row`, which is tensor-memory lane `row`.
-  const int half = warp >> 2;
+  // Worker thread (half, row): states 32 half .. 32 half + 31 of every
+  // 64-state block of row `row`, which is tensor-memory lane `row`.  Warp 8
+  // issues the MMAs.
+  const bool worker = tid < kWorkers;
+  const int half = (warp >> 2) & 1;
   const int row = (warp & 3) * 32 + (tid & 31);
   const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
   const int n = p.n, N = p.N;
@@ -189,23 +194,24 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   if (tid == 0) {
-    for (int i = 0; i < 6; ++i) mbar_init(bar_c + i, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(bar_c + i, 1);
     *abort_flag = 0;
     mbar_init_fence();
   }
   if (tid < kOnesBytes / 4) ones[tid] = 1.f;
   async_proxy_fence();  // the ones tile is read by the tensor cores
-  float cw[32];         // codewords of this thread's states
-#pragma unroll
-  for (int j = 0; j < 32; ++j) cw[j] = __ldg(p.codebook + r * kSlice + 32 * half + j);
+  if (tid < kSlice) reinterpret_cast<float*>(sm + kOffCw)[tid] = __ldg(p.codebook + r * kSlice + tid);
+  const float* cw = cws + 32 * half;  // codewords of this thread's states
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (tid == 0) mbar_arm(bar_rx, kRxBytes);
+  if (tid == 0)
+    for (int i = 0; i < kCL - 1; ++i) mbar_arm(bar_rx + i, kRxSlot);
   cluster_sync_all();  // every CTA's barriers are initialised (and armed) before any remote store
 
-  uint32_t ph_c[4] = {0, 0, 0, 0}, ph_rx = 0, ph_b = 0;
+  uint32_t ph_c[4] = {0, 0, 0, 0}, ph_b = 0;
+  uint32_t ph_rx = 0;  // parity of receive slot s in bit s
   // After one wait of this CTA gave up, no thread waits again (the call's results are void).
   auto waitb = [&](uint64_t* bar, uint32_t& ph) {
     if (!*reinterpret_cast<volatile int*>(abort_flag) && !mbar_wait(bar, ph, p.status, kDevTimeout))
@@ -267,8 +273,6 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
   auto step = [&](bool first_of_sweep, float (&y)[32]) -> float {
     tc_fence_before();
     __syncthreads();  // operand written, accumulator read: the MMAs may go
-    if (tid == 0) issue_mma(first_of_sweep);
-    __syncwarp();
     cluster_wait_plain();  // every CTA has read its receive buffer of the previous exchange
     float rs = 0.f;        // this CTA's part of the row sum
 #pragma unroll 1
@@ -288,7 +292,7 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
       }
       const uint32_t slot = static_cast<uint32_t>(r < blk ? r : r - 1);
       const uint32_t dst = mapa_u32(smem_u32(Rx) + slot * kRxSlot, static_cast<uint32_t>(blk));
-      const uint32_t rbar = mapa_u32(smem_u32(bar_rx), static_cast<uint32_t>(blk));
+      const uint32_t rbar = mapa_u32(smem_u32(bar_rx + slot), static_cast<uint32_t>(blk));
 #pragma unroll
       for (int g = 0; g < 8; ++g)
         st_async_v4f32(dst + static_cast<uint32_t>(((8 * half + g) * kMR + row) * 16), __uint_as_float(v[4 * g]),
@@ -296,26 +300,30 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
                        rbar);
       if (half == 0) st_async_f32(dst + kRxData + static_cast<uint32_t>(row * 4), rs, rbar);
     }
-    waitb(bar_c + kCL - 1, ph_c[kCL - 1]);  // the last commit: every MMA of the step is done
-    tc_fence_after();
-    {
-      uint32_t v[32];
-      tmem_ld32_async(tmem + lane_off + static_cast<uint32_t>(r * kSlice + 32 * half), v);
-      tmem_wait_ld();
+    // Received halves: added as they land, in the order the senders finish
+    // them (CTA r - 1 computes this CTA's block first); the own block's
+    // partial sums come from the last commit.
 #pragma unroll
-      for (int j = 0; j < 32; ++j) y[j] = __uint_as_float(v[j]);
-    }
-    tc_fence_before();
-    waitb(bar_rx, ph_rx);
-    if (tid == 0) mbar_arm(bar_rx, kRxBytes);  // the next exchange's phase
-    float s = 0.f;
+    for (int j = 0; j < 32; ++j) y[j] = 0.f;
 #pragma unroll 1
-    for (int src = 0; src < kCL; ++src) {
-      if (src == r) {
-        s += rs;
-        continue;
+    for (int i = 0; i < kCL - 1; ++i) {
+      if (i == kCL - 2) {
+        waitb(bar_c + kCL - 1, ph_c[kCL - 1]);  // the last commit: every MMA of the step is done
+        tc_fence_after();
+        uint32_t v[32];
+        tmem_ld32_async(tmem + lane_off + static_cast<uint32_t>(r * kSlice + 32 * half), v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) y[j] += __uint_as_float(v[j]);
+        tc_fence_before();
       }
-      const unsigned char* slot = Rx + (src < r ? src : src - 1) * kRxSlot;
+      const int src = (r + kCL - 1 - i) & (kCL - 1);
+      const int sl = src < r ? src : src - 1;
+      uint32_t ph = (ph_rx >> sl) & 1u;
+      waitb(bar_rx + sl, ph);
+      ph_rx ^= 1u << sl;
+      if (tid == 0) mbar_arm(bar_rx + sl, kRxSlot);  // the next exchange's phase
+      const unsigned char* slot = Rx + sl * kRxSlot;
 #pragma unroll
       for (int g = 0; g < 8; ++g) {
         const float4 q4 = *reinterpret_cast<const float4*>(slot + ((8 * half + g) * kMR + row) * 16);
@@ -324,10 +332,24 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
         y[4 * g + 2] += q4.z;
         y[4 * g + 3] += q4.w;
       }
-      s += *reinterpret_cast<const float*>(slot + kRxData + row * 4);
     }
+    float s = 0.f;
+#pragma unroll
+    for (int src = 0; src < kCL; ++src)
+      s += src == r ? rs : *reinterpret_cast<const float*>(Rx + (src < r ? src : src - 1) * kRxSlot + kRxData + row * 4);
     cluster_arrive_relaxed();  // this CTA's receive buffer is read
     return s;
+  };
+  // The issuing warp's part of a sweep: the n - 1 steps' barriers and MMAs.
+  auto issuer_sweep = [&]() {
+    for (int t = 1; t < n; ++t) {
+      tc_fence_before();
+      __syncthreads();  // pairs with the workers' operand barrier
+      if ((tid & 31) == 0) issue_mma(t == 1);
+      __syncwarp();
+      cluster_wait_plain();
+      cluster_arrive_relaxed();
+    }
   };
   // The next MMA's operand A: this thread's 32 values as tf32 head and tail.
   auto put_operand = [&](const float (&v)[32]) {
@@ -335,7 +357,7 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       float fh, fl;
-      split_tf32(v[j], fh, fl);
+      split_tf32_int(v[j], fh, fl);
       h[j] = __float_as_uint(fh);
       l[j] = __float_as_uint(fl);
     }
@@ -360,9 +382,10 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
     if (n > 1) load_b(p.Bfwd);  // one step has no contraction
     cluster_arrive_relaxed();   // pairs with the first step's wait
     double lsc = 0.0;           // log2 Z of the row: the references and log2 of the row sums
+    if (!worker) issuer_sweep();
     float wn = __ldg(p.w + qb), mn = __ldg(p.mtab + qb);  // the step's weight and reference, loaded a step ahead
     float ps = 0.f;                                       // this thread's part of the current vector's row sum
-    for (int t = 0; t < n; ++t) {
+    for (int t = 0; t < n && worker; ++t) {
       float y[32];
       float sprev = 1.f;
       if (t > 0) sprev = step(t == 1, y);
@@ -387,16 +410,17 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
       if (t + 1 < n) put_operand(y);
     }
     // For log Z: the last vector's row sum, by CTA and half, in the row after the partial sums.
-    ptbase[static_cast<size_t>(n) * 4 * kMR + row * 2 + half] = ps;
+    if (worker) ptbase[static_cast<size_t>(n) * 4 * kMR + row * 2 + half] = ps;
     cluster_wait_plain();  // pairs with the last arrive
     cluster_sync_all();    // every CTA is done with the forward sweep's exchanges
 
     // ---------------- backward sweep ----------------
     if (n > 1) load_b(p.Bbwd);
     cluster_arrive_relaxed();
+    if (!worker) issuer_sweep();
     wn = __ldg(p.w + qb + n - 1);
     mn = __ldg(p.mtab + qb + n - 1);
-    for (int t = n - 1; t >= 0; --t) {
+    for (int t = n - 1; t >= 0 && worker; --t) {
       float z[32];
       float4 x4[8];  // the stored forward vector of the step, requested before the exchange
 #pragma unroll
@@ -441,7 +465,7 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
     cluster_sync_all();  // every CTA's partial sums (and marginal rows) are written
 
     // log Z (CTA 0, half 0): the forward references and row sums, and the last row sum over all states.
-    if (r == 0 && half == 0 && act) {
+    if (r == 0 && worker && half == 0 && act) {
       float s = 0.f;
 #pragma unroll
       for (int src = 0; src < kCL; ++src)
@@ -455,7 +479,7 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
     }
     // Soft codeword: CTA r takes the steps t = r, r + 4, ...; the partial sums
     // over the 8 state blocks are added in a fixed order.
-    for (int t = r + kCL * (tid >> 7); t < n; t += 2 * kCL) {
+    for (int t = r + kCL * (tid >> 7); t < n && worker; t += 2 * kCL) {
       const int rr = tid & (kMR - 1);
       const int qq = tile * kMR + rr;
       if (qq >= N) continue;
@@ -473,7 +497,7 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
       p.w_hat[static_cast<size_t>(qq) * n + t] = num / den;
     }
     // Marginals: this CTA's 64 states of every step, divided by the step's sum.
-    if (p.marginals) {
+    if (p.marginals && worker) {
       for (int t = tid >> 7; t < n; t += 2) {
         const int rr = tid & (kMR - 1);
         const int qq = tile * kMR + rr;

@@ -68,6 +68,14 @@ __device__ __forceinline__ void split_tf32(float x, float& hi, float& lo) {
   lo = x - hi;
 }
 
+// The same split for finite x with integer arithmetic (add half a tf32 unit in
+// the last place to the magnitude bits, then clear the low 13 bits: round to
+// nearest, ties away from zero): keeps per-step splits off the conversion pipe.
+__device__ __forceinline__ void split_tf32_int(float x, float& hi, float& lo) {
+  hi = __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
+  lo = x - hi;
+}
+
 #define BCJR_TC_R32(r)                                                                                       \
   "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),    \
       "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),       \
