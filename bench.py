@@ -105,6 +105,23 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
+    def wait_first(self, timeout_s: float = 60.0):
+        """Block until the sampler has written its first sample, so that its
+        start-up (which can hold the driver for seconds on a fresh machine)
+        stays out of the timed region."""
+        if self.proc is None:
+            return
+        t0 = time.time()
+        while time.time() - t0 < timeout_s and self.proc.poll() is None:
+            self.f.flush()
+            try:
+                with open(self.path) as fh:
+                    if fh.readline().count(",") >= 8:
+                        return
+            except OSError:
+                pass
+            time.sleep(0.05)
+
     def stop(self):
         if self.proc is None:
             return None
@@ -216,6 +233,7 @@ def load_peaks():
 FB_SOURCES = ("fb_", "bcjr_device", "team", "bcjr_internal", "bcjr_common")
 VITERBI_SOURCES = ("viterbi_kernel", "bitshift_kernels", "bcjr_device", "team", "bcjr_internal", "bcjr_common")
 DENSE_SOURCES = ("dense_kernel", "dense_internal", "bcjr_device", "bcjr_common")
+DENSE_TC_SOURCES = ("dense_tc_kernel", "tc_util", "dense_internal", "bcjr_device", "bcjr_common")
 
 
 def kernel_source_hash(prefixes=FB_SOURCES):
@@ -298,6 +316,7 @@ def run_gpu(args):
     # ---- device-timed region: inputs resident in HBM ----
     sampler = ClockSampler(local)
     sampler.start()
+    sampler.wait_first()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     start = torch.cuda.Event(enable_timing=True)
@@ -501,6 +520,7 @@ def run_dense(args):
     barrier()
     sampler = ClockSampler(local)
     sampler.start()
+    sampler.wait_first()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     barrier()
     for i in range(args.steps):
@@ -567,6 +587,7 @@ def run_dense(args):
         sms = torch.cuda.get_device_properties(dev).multi_processor_count
         max_mhz = float(peaks.get("sm_max_mhz", 1965.0))
         fp32_peak = 2 * FP32_FMA_PER_CLK_PER_SM * sms * max_mhz * 1e6     # FLOP/s
+        tf32_peak = float(peaks.get("bf16_tflops", 1590.0)) * 1e12 * 1.1 / 2.25
         bwd_s = statistics.mean(bwd_ms) / 1e3
         fwd_s = statistics.mean(fwd_ms) / 1e3
         # the SIMT roofline is the adjoint kernel's: without the dL/dLambda extras
@@ -583,8 +604,18 @@ def run_dense(args):
                              "adjoint_dram_bytes_per_launch"), N, W["n_seq"]),
                          "kernel": "dense_fb_kernel<adjoint> (bcjr_dense_backward)",
                          "peak_source": f"2 x {FP32_FMA_PER_CLK_PER_SM} FMA/clk/SM x {sms} SMs x {max_mhz:.0f} MHz"},
+            # the forward call's contraction runs on the tensor cores (three tf32
+            # products per step): against the tf32 peak, the measured bf16 GEMM
+            # rate times the nominal tf32 / bf16 ratio (1.1 / 2.25 PFLOP/s dense)
             "forward_call": {"ms": 1e3 * fwd_s, "TFLOP/s": flops_f / fwd_s / 1e12,
-                             "frac": flops_f / fwd_s / fp32_peak},
+                             "kernel": "dense_tc_fwd_kernel (tcgen05.mma kind::tf32, three products)",
+                             "bound": "tensor", "peak": tf32_peak / 1e12,
+                             "frac": flops_f / fwd_s / tf32_peak,
+                             "frac_executed_3xtf32": 3 * flops_f / fwd_s / tf32_peak,
+                             "peak_source": "measured bf16 GEMM x 1.1 / 2.25 (nominal tf32 / bf16 dense)",
+                             "traffic": scaled_traffic(load_traffic("dense_tc_fwd_kernel_S256_slice.md",
+                                                                   DENSE_TC_SOURCES).get("fwd_dram_bytes_per_launch"),
+                                                       N, W["n_seq"])},
             "kernels_ms": {"bcjr_dense_forward": 1e3 * fwd_s,
                            ("bcjr_dense_backward_lambda" if wl else "bcjr_dense_backward"): 1e3 * bwd_s},
             "gpu_launches": (7 if wl else 5) * args.steps,  # prep + forward; prep + adjoint + reduction (+ tensor-core sum + reduction)
@@ -650,6 +681,7 @@ def run_viterbi(args):
     barrier()
     sampler = ClockSampler(local)
     sampler.start()
+    sampler.wait_first()
     s0, e0 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     s0.record(stream)
@@ -757,6 +789,7 @@ def run_bitwidth(args):
     mufu_peak = MUFU_OPS_PER_CLK_PER_SM * sms * max_mhz * 1e6
     sampler = ClockSampler(local)
     sampler.start()
+    sampler.wait_first()
     per_k = {}
     for k in W["k"]:
         ws_f, ws_b, ws_v = B.Workspace(dev), B.Workspace(dev), B.Workspace(dev)

@@ -539,13 +539,22 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
 // ---------------------------------------------------------------------------
 size_t dense_tc_smem_bytes() { return dtc::kSmemBytes; }
 
-int dense_tc_max_clusters() {
+namespace {
+// Per device: the kernel's shared-memory attribute is set and its cluster
+// occupancy queried once, so that later calls issue no driver queries (a
+// query can wait behind other users of the driver).  0 = not yet known.
+constexpr int kMaxDevices = 64;
+int g_tc_clusters[kMaxDevices] = {};
+
+int tc_clusters_of_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
+  if (dev < kMaxDevices && g_tc_clusters[dev] > 0) return g_tc_clusters[dev];
   const size_t smem = dense_tc_smem_bytes();
   if (cudaFuncSetAttribute(dense_tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
       cudaSuccess)
     return 0;
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(dtc::kCL * sms, 1, 1);
@@ -553,8 +562,12 @@ int dense_tc_max_clusters() {
   cfg.dynamicSmemBytes = smem;
   int clusters = 0;
   if (cudaOccupancyMaxActiveClusters(&clusters, dense_tc_fwd_kernel, &cfg) != cudaSuccess) return 0;
+  if (dev < kMaxDevices) g_tc_clusters[dev] = clusters;
   return clusters;
 }
+}  // namespace
+
+int dense_tc_max_clusters() { return tc_clusters_of_device(); }
 
 cudaError_t launch_dense_tc_forward(const DenseTCParams& p, const float* lam, int clusters, cudaStream_t s) {
   using namespace dtc;
@@ -566,11 +579,8 @@ cudaError_t launch_dense_tc_forward(const DenseTCParams& p, const float* lam, in
   dense_tc_mtab_kernel<<<static_cast<unsigned>(blocks < 4096 ? blocks : 4096), kS, 0, s>>>(p.w, p.codebook, p.sc2, total,
                                                                                          p.mtab);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const size_t smem = dense_tc_smem_bytes();
-  if ((e = cudaFuncSetAttribute(dense_tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(smem))) != cudaSuccess)
-    return e;
-  dense_tc_fwd_kernel<<<clusters * kCL, kThreads, smem, s>>>(p);
+  if (tc_clusters_of_device() < 1) return cudaErrorNotSupported;  // also sets the shared-memory attribute
+  dense_tc_fwd_kernel<<<clusters * kCL, kThreads, dense_tc_smem_bytes(), s>>>(p);
   return cudaGetLastError();
 }
 
