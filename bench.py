@@ -44,7 +44,7 @@ MUFU_OPS_PER_CLK_PER_SM = 16      # ex2/lg2 throughput per SM per clock (compute
 FP32_FMA_PER_CLK_PER_SM = 128     # float32 fma lanes per SM per clock (compute capability 10.0)
 FP64_OPS_PER_CLK_PER_SM = 64     # float64 lanes per SM per clock (compute capability 10.0)
 VITERBI_METRIC = "Viterbi hard decode weights/s at S=2^16,k=2 (2048x8192 projection); % of FP64 peak"
-DENSE_METRIC = "dense BCJR fwd+bwd weights/s at S=256, n=4096, N=4096; % of FP32 peak"
+DENSE_METRIC = "dense BCJR fwd+bwd weights/s at S=256, n=4096, N=4096; % of tf32 tensor peak"
 DENSE_WORKLOAD = "dense_S256"
 ALG_MUFU_PER_STATE_STEP = 4       # one forward and one backward log-sum-exp in each of the two calls
 
@@ -232,7 +232,6 @@ def load_peaks():
 # Sources that define each measured kernel (its ncu counters go stale when they change).
 FB_SOURCES = ("fb_", "bcjr_device", "team", "bcjr_internal", "bcjr_common")
 VITERBI_SOURCES = ("viterbi_kernel", "bitshift_kernels", "bcjr_device", "team", "bcjr_internal", "bcjr_common")
-DENSE_SOURCES = ("dense_kernel", "dense_internal", "bcjr_device", "bcjr_common")
 DENSE_TC_SOURCES = ("dense_tc_kernel", "tc_util", "dense_internal", "bcjr_device", "bcjr_common")
 
 
@@ -590,7 +589,7 @@ def run_dense(args):
         tf32_peak = float(peaks.get("bf16_tflops", 1590.0)) * 1e12 * 1.1 / 2.25
         bwd_s = statistics.mean(bwd_ms) / 1e3
         fwd_s = statistics.mean(fwd_ms) / 1e3
-        # the SIMT roofline is the adjoint kernel's: without the dL/dLambda extras
+        # the roofline is the plain adjoint kernel's: without the dL/dLambda extras
         adj_s = plain_bwd_ms / 1e3 if wl else bwd_s
         flops_b = 2 * 4 * N * n * S * S   # adjoint: two stacked contractions per sweep, two sweeps
         flops_f = 2 * 2 * N * n * S * S   # forward call: one contraction per sweep, two sweeps
@@ -598,15 +597,19 @@ def run_dense(args):
             "metric": DENSE_METRIC, "value": value, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": _dense_config(world, N),
-            "roofline": {"bound": "alu", "pipe": "FP32 FMA (SIMT)", "achieved": flops_b / adj_s / 1e12,
-                         "peak": fp32_peak / 1e12, "unit": "TFLOP/s", "frac": flops_b / adj_s / fp32_peak,
-                         "traffic": scaled_traffic(load_traffic("dense_fb_kernel_S256_full.md", DENSE_SOURCES).get(
-                             "adjoint_dram_bytes_per_launch"), N, W["n_seq"]),
-                         "kernel": "dense_fb_kernel<adjoint> (bcjr_dense_backward)",
-                         "peak_source": f"2 x {FP32_FMA_PER_CLK_PER_SM} FMA/clk/SM x {sms} SMs x {max_mhz:.0f} MHz"},
-            # the forward call's contraction runs on the tensor cores (three tf32
-            # products per step): against the tf32 peak, the measured bf16 GEMM
-            # rate times the nominal tf32 / bf16 ratio (1.1 / 2.25 PFLOP/s dense)
+            # Both calls run their per-step contractions on the tensor cores (three
+            # tf32 products per step).  The peak is the tf32 rate: the measured
+            # bf16 GEMM rate times the nominal tf32 / bf16 ratio (1.1 / 2.25 PFLOP/s
+            # dense); `achieved` counts the algorithmic contraction (one product).
+            "roofline": {"bound": "tensor", "achieved": flops_b / adj_s / 1e12, "peak": tf32_peak / 1e12,
+                         "unit": "TFLOP/s", "frac": flops_b / adj_s / tf32_peak,
+                         "frac_executed_3xtf32": 3 * flops_b / adj_s / tf32_peak,
+                         "traffic": scaled_traffic(load_traffic("dense_tc_adj_kernel_S256_slice.md",
+                                                                DENSE_TC_SOURCES).get("bwd_dram_bytes_per_launch"),
+                                                   N, W["n_seq"]),
+                         "kernel": "dense_tc_kernel<adjoint> (bcjr_dense_backward; tcgen05.mma kind::tf32)",
+                         "peak_source": "measured bf16 GEMM x 1.1 / 2.25 (nominal tf32 / bf16 dense)",
+                         "fp32_simt_peak": fp32_peak / 1e12},
             "forward_call": {"ms": 1e3 * fwd_s, "TFLOP/s": flops_f / fwd_s / 1e12,
                              "kernel": "dense_tc_fwd_kernel (tcgen05.mma kind::tf32, three products)",
                              "bound": "tensor", "peak": tf32_peak / 1e12,
@@ -618,7 +621,9 @@ def run_dense(args):
                                                        N, W["n_seq"])},
             "kernels_ms": {"bcjr_dense_forward": 1e3 * fwd_s,
                            ("bcjr_dense_backward_lambda" if wl else "bcjr_dense_backward"): 1e3 * bwd_s},
-            "gpu_launches": (7 if wl else 5) * args.steps,  # prep + forward; prep + adjoint + reduction (+ tensor-core sum + reduction)
+            # forward: prep, reference, kernel; backward: prep, reference, kernel, codebook reduction
+            # (with dL/dLambda: prep, adjoint, codebook reduction, row-product sum, reduction)
+            "gpu_launches": (3 + (5 if wl else 4)) * args.steps,
             "clocks": clocks,
         }
         if wl:

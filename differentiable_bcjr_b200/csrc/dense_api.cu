@@ -18,9 +18,11 @@ struct DenseLayout {
   size_t P, PT, ckx, ckf, ckv, ckw, mtab, gc, dlpart, total, ck_stride, mt_stride;
 };
 
-// `dl_parts` > 0 adds the rows V, W of the log-transition gradient and that
-// many [S][S] partial sums.
-DenseLayout dense_layout(int grid, int n, bool adjoint, int dl_parts = 0) {
+// Workspace of the vector-Jacobian product with the log-transition gradient:
+// P and P^T, per CTA the rows X, U, V, W of that gradient (X and U in the
+// places of the stored forward values) and the step references, the codebook
+// partials, and `dl_parts` [S][S] partial sums of the row products.
+DenseLayout dense_layout(int grid, int n, int dl_parts) {
   const size_t S = bcjr::kDenseStates, M = bcjr::kDenseRows;
   DenseLayout l = {};
   l.ck_stride = static_cast<size_t>(n) * M * S;
@@ -34,33 +36,37 @@ DenseLayout dense_layout(int grid, int n, bool adjoint, int dl_parts = 0) {
   l.ckx = off;
   off = align_up(off + ck_bytes);
   l.ckf = off;
-  if (adjoint) off = align_up(off + ck_bytes);
+  off = align_up(off + ck_bytes);
   l.ckv = off;
-  if (dl_parts > 0) off = align_up(off + ck_bytes);
+  off = align_up(off + ck_bytes);
   l.ckw = off;
-  if (dl_parts > 0) off = align_up(off + ck_bytes);
+  off = align_up(off + ck_bytes);
   l.mtab = off;
   off = align_up(off + static_cast<size_t>(grid) * l.mt_stride * sizeof(float));
   l.gc = off;
-  if (adjoint) off = align_up(off + static_cast<size_t>(grid) * S * sizeof(float));
+  off = align_up(off + static_cast<size_t>(grid) * S * sizeof(float));
   l.dlpart = off;
   off = align_up(off + static_cast<size_t>(dl_parts) * S * S * sizeof(float));
   l.total = off;
   return l;
 }
 
-// Workspace of the forward call (tensor cores): the transfer matrix as two
-// sets of resident operand slices, the emission reference of every step, and
-// per CTA of the resident clusters its forward vectors and partial sums.
+// Workspace of the tensor-core calls: the transfer matrix as two sets of
+// resident operand slices, the emission reference of every step, and per CTA
+// of the resident clusters its stored forward values and partial sums (the
+// adjoint adds the F~ ratios, the forward row sums and the codebook-gradient
+// partials of each cluster).
 struct DenseTCLayout {
-  size_t Bfwd, Bbwd, mtab, ck, part, total, ck_stride, part_stride;
+  size_t Bfwd, Bbwd, mtab, ck, ckf, cks, part, gc, total, ck_stride, cks_stride, part_stride;
 };
 
-DenseTCLayout dense_tc_layout(int clusters, int n, int N) {
-  const size_t S = bcjr::kDenseStates, R = bcjr::kDenseTCRows, CL = bcjr::kDenseTCCluster;
+DenseTCLayout dense_tc_layout(bool adjoint, int clusters, int n, int N) {
+  const size_t S = bcjr::kDenseStates, CL = bcjr::kDenseTCCluster;
+  const size_t seqs = static_cast<size_t>(bcjr::dense_tc_tile_seqs(adjoint));
   DenseTCLayout l = {};
-  l.ck_stride = static_cast<size_t>(n) * R * (S / CL);
-  l.part_stride = static_cast<size_t>(2 * n + 1) * R * 2;
+  l.ck_stride = static_cast<size_t>(n) * seqs * (S / CL);
+  l.cks_stride = adjoint ? static_cast<size_t>(n) * seqs : 0;
+  l.part_stride = adjoint ? static_cast<size_t>(n + 2) * 4 * seqs : static_cast<size_t>(2 * n + 1) * seqs * 2;
   const size_t ctas = static_cast<size_t>(clusters) * CL;
   size_t off = kHeader;
   l.Bfwd = off;
@@ -71,16 +77,23 @@ DenseTCLayout dense_tc_layout(int clusters, int n, int N) {
   off = align_up(off + static_cast<size_t>(N) * n * sizeof(float));
   l.ck = off;
   off = align_up(off + ctas * l.ck_stride * sizeof(float));
+  l.ckf = off;
+  if (adjoint) off = align_up(off + ctas * l.ck_stride * sizeof(float));
+  l.cks = off;
+  off = align_up(off + ctas * l.cks_stride * sizeof(float));
   l.part = off;
   off = align_up(off + ctas * l.part_stride * sizeof(float));
+  l.gc = off;
+  if (adjoint) off = align_up(off + static_cast<size_t>(clusters) * S * sizeof(float));
   l.total = off;
   return l;
 }
 
-bcjr_status dense_tc_clusters(int N, int* clusters) {
-  const int cap = bcjr::dense_tc_max_clusters();
+bcjr_status dense_tc_clusters(bool adjoint, int N, int* clusters) {
+  const int cap = bcjr::dense_tc_max_clusters(adjoint);
   if (cap < 1) return BCJR_ERR_UNSUPPORTED;
-  const int tiles = (N + bcjr::kDenseTCRows - 1) / bcjr::kDenseTCRows;
+  const int per = bcjr::dense_tc_tile_seqs(adjoint);
+  const int tiles = (N + per - 1) / per;
   *clusters = tiles < 1 ? 1 : (tiles < cap ? tiles : cap);
   return BCJR_OK;
 }
@@ -91,7 +104,7 @@ bcjr_status dense_tc_clusters(int N, int* clusters) {
 // of 32 x (CTAs that fit) sequences.  `parts` = partial sums of the reduction
 // (one per SM).
 bcjr_status dlam_geometry(int N, int* grid, int* chunk, int* parts) {
-  const int cap = bcjr::dense_max_grid(true);
+  const int cap = bcjr::dense_max_grid();
   if (cap < 1) return BCJR_ERR_UNSUPPORTED;
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
@@ -144,41 +157,49 @@ bcjr_status dense_common(bool adjoint, const float* g, const float* w, const flo
     if (marginals && !aligned(marginals, 16)) return BCJR_ERR_INVALID_ARG;
   }
   if (!ws || !aligned(ws, kAlign)) return BCJR_ERR_WORKSPACE;
-  if (!adjoint) {
-    // The soft codeword: the tensor-core kernel (dense_tc_kernel.cu).
+  if (!grad_lam) {
+    // The soft codeword and the plain vector-Jacobian product: the tensor-core
+    // kernels (dense_tc_kernel.cu).
     int clusters = 0;
-    if ((st = dense_tc_clusters(N, &clusters)) != BCJR_OK) return st;
-    const DenseTCLayout lt = dense_tc_layout(clusters, n, N);
+    if ((st = dense_tc_clusters(adjoint, N, &clusters)) != BCJR_OK) return st;
+    const DenseTCLayout lt = dense_tc_layout(adjoint, clusters, n, N);
     if (ws_bytes < lt.total) return BCJR_ERR_WORKSPACE;
     char* b = static_cast<char*>(ws);
     bcjr::DenseTCParams tp = {};
     tp.w = w;
     tp.codebook = c;
+    tp.g = g;
+    tp.what_in = what_in;
     tp.mtab = reinterpret_cast<float*>(b + lt.mtab);
     tp.Bfwd = reinterpret_cast<float*>(b + lt.Bfwd);
     tp.Bbwd = reinterpret_cast<float*>(b + lt.Bbwd);
     tp.ck = reinterpret_cast<float*>(b + lt.ck);
+    tp.ckf = reinterpret_cast<float*>(b + lt.ckf);
+    tp.cks = reinterpret_cast<float*>(b + lt.cks);
     tp.part = reinterpret_cast<float*>(b + lt.part);
+    tp.gc_part = reinterpret_cast<float*>(b + lt.gc);
     tp.w_hat = w_hat;
     tp.marginals = marginals;
     tp.log_z = log_z;
+    tp.grad_w = grad_w;
     tp.status = reinterpret_cast<int*>(b);
     tp.ck_stride = lt.ck_stride;
+    tp.cks_stride = lt.cks_stride;
     tp.part_stride = lt.part_stride;
     tp.sc2 = static_cast<float>(1.4426950408889634 / static_cast<double>(T));
+    tp.two_over_T = static_cast<float>(2.0 / static_cast<double>(T));
     tp.n = n;
     tp.N = N;
     if ((st = from_cuda(cudaMemsetAsync(ws, 0, sizeof(int), s))) != BCJR_OK) return st;
-    return from_cuda(bcjr::launch_dense_tc_forward(tp, lam, clusters, s));
+    if ((st = from_cuda(bcjr::launch_dense_tc(tp, lam, adjoint, clusters, s))) != BCJR_OK) return st;
+    if (adjoint) return from_cuda(bcjr::launch_gradc_reduce(tp.gc_part, clusters, S, grad_c, accumulate, s));
+    return BCJR_OK;
   }
-  const bool dl = adjoint && grad_lam;
+  // The vector-Jacobian product with the log-transition gradient (SIMT kernel
+  // writing full-width rows for the tensor-core row-product sum).
   int grid = 0, chunk = N, parts = 0;
-  if (dl) {
-    if ((st = dlam_geometry(N, &grid, &chunk, &parts)) != BCJR_OK) return st;
-  } else if ((st = from_cuda(bcjr::dense_geometry(adjoint, N, &grid))) != BCJR_OK) {
-    return st;
-  }
-  const DenseLayout lay = dense_layout(grid, n, adjoint, parts);
+  if ((st = dlam_geometry(N, &grid, &chunk, &parts)) != BCJR_OK) return st;
+  const DenseLayout lay = dense_layout(grid, n, parts);
   if (ws_bytes < lay.total) return BCJR_ERR_WORKSPACE;
   char* base = static_cast<char*>(ws);
   bcjr::DenseParams p = {};
@@ -195,8 +216,8 @@ bcjr_status dense_common(bool adjoint, const float* g, const float* w, const flo
   p.PT = reinterpret_cast<const float*>(base + lay.PT);
   p.ckx = reinterpret_cast<float*>(base + lay.ckx);
   p.ckf = reinterpret_cast<float*>(base + lay.ckf);
-  p.ckv = dl ? reinterpret_cast<float*>(base + lay.ckv) : nullptr;
-  p.ckw = dl ? reinterpret_cast<float*>(base + lay.ckw) : nullptr;
+  p.ckv = reinterpret_cast<float*>(base + lay.ckv);
+  p.ckw = reinterpret_cast<float*>(base + lay.ckw);
   p.mtab = reinterpret_cast<float*>(base + lay.mtab);
   p.status = reinterpret_cast<int*>(base);
   p.ck_stride = lay.ck_stride;
@@ -206,11 +227,6 @@ bcjr_status dense_common(bool adjoint, const float* g, const float* w, const flo
   p.n = n;
   p.N = N;
   if ((st = from_cuda(cudaMemsetAsync(ws, 0, sizeof(int), s))) != BCJR_OK) return st;
-  if (!dl) {
-    if ((st = from_cuda(bcjr::launch_dense(p, lam, adjoint, grid, s))) != BCJR_OK) return st;
-    if (adjoint) return from_cuda(bcjr::launch_gradc_reduce(p.gc_part, grid, S, grad_c, accumulate, s));
-    return BCJR_OK;
-  }
   // Backward call with the log-transition gradient, chunk by chunk: each
   // chunk's backward kernel writes the rows X, U, V, W of its transitions, the
   // tensor-core kernel sums them into per-SM partials, and the reductions add
@@ -227,7 +243,7 @@ bcjr_status dense_common(bool adjoint, const float* g, const float* w, const flo
     pc.grad_w = grad_w + off;
     pc.N = Nc;
     const int grid_c = (Nc + bcjr::kDenseRows - 1) / bcjr::kDenseRows;
-    if ((st = from_cuda(bcjr::launch_dense(pc, lam, true, grid_c, s, c0 == 0))) != BCJR_OK) return st;
+    if ((st = from_cuda(bcjr::launch_dense(pc, lam, grid_c, s, c0 == 0))) != BCJR_OK) return st;
     if ((st = from_cuda(bcjr::launch_gradc_reduce(pc.gc_part, grid_c, S, grad_c, acc, s))) != BCJR_OK) return st;
     if (n == 1) {  // no transitions: the gradient is zero
       if (!acc && (st = from_cuda(cudaMemsetAsync(grad_lam, 0, S * S * sizeof(float), s))) != BCJR_OK) return st;
@@ -262,15 +278,11 @@ size_t bcjr_dense_workspace_size_impl(int op, int n_states, int seq_len, int n_s
   if (op == BCJR_OP_DENSE_BACKWARD_LAMBDA) {
     int chunk = 0, parts = 0;
     if (dlam_geometry(n_seq > 0 ? n_seq : 1, &grid, &chunk, &parts) != BCJR_OK) return 0;
-    return dense_layout(grid, seq_len, true, parts).total;
+    return dense_layout(grid, seq_len, parts).total;
   }
-  if (!adjoint) {
-    int clusters = 0;
-    if (dense_tc_clusters(n_seq > 0 ? n_seq : 1, &clusters) != BCJR_OK) return 0;
-    return dense_tc_layout(clusters, seq_len, n_seq > 0 ? n_seq : 1).total;
-  }
-  if (bcjr::dense_geometry(adjoint, n_seq > 0 ? n_seq : 1, &grid) != cudaSuccess) return 0;
-  return dense_layout(grid, seq_len, adjoint).total;
+  int clusters = 0;
+  if (dense_tc_clusters(adjoint, n_seq > 0 ? n_seq : 1, &clusters) != BCJR_OK) return 0;
+  return dense_tc_layout(adjoint, clusters, seq_len, n_seq > 0 ? n_seq : 1).total;
 }
 
 extern "C" {

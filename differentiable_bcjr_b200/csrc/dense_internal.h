@@ -38,28 +38,37 @@ struct DenseParams {
   int n, N;
 };
 
-// Soft codeword of the dense trellis on the tensor cores (dense_tc_kernel.cu):
-// a cluster of kDenseTCCluster CTAs per kDenseTCRows sequences, CTA r holding
-// K-slice r of the transfer matrix.
+// The dense trellis on the tensor cores (dense_tc_kernel.cu): a cluster of
+// kDenseTCCluster CTAs per tile of kDenseTCRows MMA rows, CTA r holding K-slice
+// r of the transfer matrix.  The soft-codeword call puts one sequence on each
+// row (128 per tile); the vector-Jacobian product stacks each sequence's two
+// operands on adjacent rows (64 sequences per tile).
 constexpr int kDenseTCCluster = 4;
 constexpr int kDenseTCRows = 128;
 
 struct DenseTCParams {
   const float* w;          // [N][n]
   const float* codebook;   // [S]
+  const float* g;          // [N][n] upstream gradient (vector-Jacobian product)
+  const float* what_in;    // [N][n] soft codeword of the forward call (vector-Jacobian product)
   float* mtab;             // [N][n] emission reference of every step (written by the reference kernel)
   float* Bfwd;             // [4 slices][128 KiB] P as resident operand tiles (forward sweep)
   float* Bbwd;             // the same for P^T (backward sweep)
-  float* ck;               // per CTA [n][16][128] float4: forward vectors, this CTA's 64 states
-  float* part;             // per CTA [n][2 halves][128][2] partial sums (sum c gamma, sum gamma) over
-                           // 32 states each, then [128][2 halves] the last forward vector's row sums
-  float* w_hat;            // [N][n]
-  float* marginals;        // [N][n][S] or null
-  float* log_z;            // [N] or null
+  float* ck;               // per CTA: forward vectors of this CTA's 64 states, every step
+  float* ckf;              // per CTA: forward adjoint ratios F~ (vector-Jacobian product)
+  float* cks;              // per CTA [n][64]: every step's forward row sum (vector-Jacobian product)
+  float* part;             // per CTA: per-row partial sums over its states (layouts in the kernel)
+  float* w_hat;            // [N][n] (soft codeword)
+  float* marginals;        // [N][n][S] or null (soft codeword)
+  float* log_z;            // [N] or null (soft codeword)
+  float* grad_w;           // [N][n] (vector-Jacobian product)
+  float* gc_part;          // [clusters][S] codebook-gradient partials (vector-Jacobian product)
   int* status;
-  size_t ck_stride;        // floats per CTA in ck
+  size_t ck_stride;        // floats per CTA in ck and ckf
+  size_t cks_stride;       // floats per CTA in cks
   size_t part_stride;      // floats per CTA in part
   float sc2;               // log2(e) / T
+  float two_over_T;
   int n, N;
 };
 
@@ -78,16 +87,18 @@ struct DlamParams {
   long long total_stages;
 };
 
-// Dense launchers (dense_kernel.cu, dense_dlam_kernel.cu).
-size_t dense_smem_bytes(bool adjoint);
-cudaError_t dense_geometry(bool adjoint, int n_seq, int* grid);
-int dense_max_grid(bool adjoint);
+// Launchers of the vector-Jacobian product that also writes the rows of the
+// log-transition gradient (dense_kernel.cu) and of that gradient's row sum
+// (dense_dlam_kernel.cu).
+size_t dense_smem_bytes();
+int dense_max_grid();
 cudaError_t launch_dense_prep(const float* lam, const DenseParams& p, cudaStream_t s);
-cudaError_t launch_dense(const DenseParams& p, const float* lam, bool adjoint, int grid, cudaStream_t s,
-                         bool prep = true);
+cudaError_t launch_dense(const DenseParams& p, const float* lam, int grid, cudaStream_t s, bool prep = true);
 size_t dense_tc_smem_bytes();
-int dense_tc_max_clusters();
-cudaError_t launch_dense_tc_forward(const DenseTCParams& p, const float* lam, int clusters, cudaStream_t s);
+int dense_tc_max_clusters(bool adjoint);
+// Sequences per cluster tile: 128 for the soft codeword, 64 for the adjoint.
+constexpr int dense_tc_tile_seqs(bool adjoint) { return adjoint ? kDenseTCRows / 2 : kDenseTCRows; }
+cudaError_t launch_dense_tc(const DenseTCParams& p, const float* lam, bool adjoint, int clusters, cudaStream_t s);
 size_t dlam_smem_bytes();
 cudaError_t dlam_grid(long long total_stages, int* grid);
 cudaError_t launch_dlam(const DlamParams& p, int grid, cudaStream_t s);

@@ -1,4 +1,9 @@
-// dense_kernel.cu -- forward-backward over a dense (fully connected) trellis (sm_100a).
+// dense_kernel.cu -- vector-Jacobian product over a dense (fully connected)
+// trellis that also writes the rows of the log-transition gradient (sm_100a):
+// the kernel behind bcjr_dense_backward_lambda.  The soft codeword and the
+// plain vector-Jacobian product run on the tensor cores (dense_tc_kernel.cu);
+// this kernel keeps all 256 states of a sequence in one CTA so that it can
+// write the full-width rows X, U, V, W that dense_dlam_kernel.cu sums.
 //
 // "BCJR-QAT: A Differentiable Relaxation of Trellis-Coded Weight Quantization",
 // abstract: the relaxation is a 1D Ising-like chain solved by a transfer
@@ -45,7 +50,6 @@ constexpr int kKC = 32;           // rows of P per shared-memory window
 constexpr int kChunks = kS / kKC;
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <bool ADJ>
 struct Cfg {
   static constexpr int RQ = 4;  // sequences per thread (8 warps per CTA)
   static constexpr int WARPS = kM / RQ;
@@ -85,15 +89,14 @@ __global__ void dense_prep_kernel(const float* __restrict__ lam, float* __restri
   }
 }
 
-template <bool ADJ>
-__global__ void __launch_bounds__(dense::Cfg<ADJ>::THREADS, 1) dense_fb_kernel(const DenseParams p) {
+__global__ void __launch_bounds__(dense::Cfg::THREADS, 1) dense_adj_kernel(const DenseParams p) {
   using namespace dense;
-  constexpr int RQ = Cfg<ADJ>::RQ;
-  constexpr int NTH = Cfg<ADJ>::THREADS;
+  constexpr int RQ = Cfg::RQ;
+  constexpr int NTH = Cfg::THREADS;
   extern __shared__ __align__(16) float sm[];
   float* A1 = sm;                           // [S][M] first operand
   float* A2 = A1 + kS * kM;                 // [S][M] second operand (adjoint)
-  float* Pc = A2 + (ADJ ? kS * kM : 0);     // [2][KC][S] window of P or P^T
+  float* Pc = A2 + kS * kM;     // [2][KC][S] window of P or P^T
   float* stX = Pc + 2 * kKC * kS;           // [M][S] staged x_t (backward)
   float* stF = stX + kM * kS;               // [M][S] staged F~_t (adjoint backward)
 
@@ -110,7 +113,7 @@ __global__ void __launch_bounds__(dense::Cfg<ADJ>::THREADS, 1) dense_fb_kernel(c
   for (int j = 0; j < 8; ++j) gcacc[j] = 0.f;
 
   float* ckx = p.ckx + static_cast<size_t>(blockIdx.x) * p.ck_stride;
-  float* ckf = ADJ ? p.ckf + static_cast<size_t>(blockIdx.x) * p.ck_stride : nullptr;
+  float* ckf = p.ckf + static_cast<size_t>(blockIdx.x) * p.ck_stride;
   float* mtab = p.mtab + static_cast<size_t>(blockIdx.x) * p.mt_stride;
 
   // One 32-row window of B (P or P^T) into buffer `buf`, plus optional extra 16-byte copies.
@@ -125,12 +128,12 @@ __global__ void __launch_bounds__(dense::Cfg<ADJ>::THREADS, 1) dense_fb_kernel(c
   };
   auto issue_stage = [&](int t) {  // x_t (and F~_t) of this CTA's rows into the staging tiles
     const float* srcx = ckx + static_cast<size_t>(t) * kM * kS;
-    const float* srcf = ADJ ? ckf + static_cast<size_t>(t) * kM * kS : nullptr;
+    const float* srcf = ckf + static_cast<size_t>(t) * kM * kS;
 #pragma unroll
     for (int r = 0; r < (kM * kS) / (4 * NTH); ++r) {
       const int i = (tid + r * NTH) * 4;
       cp_async16(stX + i, srcx + i);
-      if constexpr (ADJ) cp_async16(stF + i, srcf + i);
+      cp_async16(stF + i, srcf + i);
     }
   };
 
@@ -143,7 +146,7 @@ __global__ void __launch_bounds__(dense::Cfg<ADJ>::THREADS, 1) dense_fb_kernel(c
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         acc1[i][j] = 0.f;
-        if constexpr (ADJ) acc2[i][j] = 0.f;
+        acc2[i][j] = 0.f;
       }
     for (int kc = 0; kc < kChunks; ++kc) {
       cp_async_wait<0>();
@@ -173,7 +176,7 @@ __global__ void __launch_bounds__(dense::Cfg<ADJ>::THREADS, 1) dense_fb_kernel(c
               acc1[4 * g + i][2 * j] = c2.x;
               acc1[4 * g + i][2 * j + 1] = c2.y;
             }
-          if constexpr (ADJ) {
+          {
             const float4 a2 = *reinterpret_cast<const float4*>(A2 + a_index(s, q));
             const float av2[4] = {a2.x, a2.y, a2.z, a2.w};
 #pragma unroll
@@ -241,7 +244,7 @@ __global__ void __launch_bounds__(dense::Cfg<ADJ>::THREADS, 1) dense_fb_kernel(c
         for (int j = 0; j < 8; ++j) {
           const float e = ex2f(ph[j] - m2);
           x[j] = (t > 0) ? acc1[i][j] * e : e;
-          if constexpr (ADJ) F[j] = (t > 0 && acc1[i][j] > 0.f) ? acc2[i][j] / acc1[i][j] : 0.f;
+          F[j] = (t > 0 && acc1[i][j] > 0.f) ? acc2[i][j] / acc1[i][j] : 0.f;
           sum += x[j];
         }
         const float sig = warp_sum(sum);
@@ -249,20 +252,20 @@ __global__ void __launch_bounds__(dense::Cfg<ADJ>::THREADS, 1) dense_fb_kernel(c
         lsc[i] += static_cast<double>(m2) + static_cast<double>(log2f(sig));
         float eps[8];
         float gt = 0.f, wh = 0.f;
-        if constexpr (ADJ) {
+        {
           gt = load_row(p.g, i, t);
           wh = load_row(p.what_in, i, t);
         }
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           x[j] *= inv;
-          if constexpr (ADJ) eps[j] = gt * (cs[j] - wh);
+          eps[j] = gt * (cs[j] - wh);
         }
         if (lane == 0) mtab[static_cast<size_t>(t) * kM + q] = m2;
         float* cx = ckx + (static_cast<size_t>(t) * kM + q) * kS;
         *reinterpret_cast<float4*>(cx + 4 * lane) = make_float4(x[0], x[1], x[2], x[3]);
         *reinterpret_cast<float4*>(cx + 128 + 4 * lane) = make_float4(x[4], x[5], x[6], x[7]);
-        if constexpr (ADJ) {
+        {
           float* cf = ckf + (static_cast<size_t>(t) * kM + q) * kS;
           *reinterpret_cast<float4*>(cf + 4 * lane) = make_float4(F[0], F[1], F[2], F[3]);
           *reinterpret_cast<float4*>(cf + 128 + 4 * lane) = make_float4(F[4], F[5], F[6], F[7]);
@@ -271,9 +274,9 @@ __global__ void __launch_bounds__(dense::Cfg<ADJ>::THREADS, 1) dense_fb_kernel(c
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             A1[a_index(st_of(lane, j), q)] = x[j];
-            if constexpr (ADJ) A2[a_index(st_of(lane, j), q)] = x[j] * (F[j] + eps[j]);
+            A2[a_index(st_of(lane, j), q)] = x[j] * (F[j] + eps[j]);
           }
-        } else if constexpr (ADJ) {
+        } else {
           // D = E[sum_u eps_u] = sum_s gamma_{n-1}(s) (F~_{n-1}(s) + eps_{n-1}(s)); z_{n-1} = 1
           float dsum = 0.f;
 #pragma unroll
@@ -282,22 +285,10 @@ __global__ void __launch_bounds__(dense::Cfg<ADJ>::THREADS, 1) dense_fb_kernel(c
         }
       }
     }
-    if constexpr (!ADJ) {
-      if (lane == 0) {
+    if (lane == 0) {
 #pragma unroll
-        for (int i = 0; i < RQ; ++i) {
-          if (!act[i]) continue;
-          const double lz = lsc[i] * 0.69314718055994530942;
-          if (!isfinite(lz)) atomicOr(p.status, kDevNonFinite);
-          if (p.log_z) p.log_z[qg[i]] = static_cast<float>(lz);
-        }
-      }
-    } else {
-      if (lane == 0) {
-#pragma unroll
-        for (int i = 0; i < RQ; ++i)
-          if (act[i] && !(isfinite(lsc[i]) && isfinite(Dv[i]))) atomicOr(p.status, kDevNonFinite);
-      }
+      for (int i = 0; i < RQ; ++i)
+        if (act[i] && !(isfinite(lsc[i]) && isfinite(Dv[i]))) atomicOr(p.status, kDevNonFinite);
     }
 
     // ---------------- backward sweep ----------------
@@ -317,7 +308,7 @@ __global__ void __launch_bounds__(dense::Cfg<ADJ>::THREADS, 1) dense_fb_kernel(c
           const float4 x1 = *reinterpret_cast<const float4*>(stX + q * kS + 128 + 4 * lane);
           x[0] = x0.x; x[1] = x0.y; x[2] = x0.z; x[3] = x0.w;
           x[4] = x1.x; x[5] = x1.y; x[6] = x1.z; x[7] = x1.w;
-          if constexpr (ADJ) {
+          {
             const float4 f0 = *reinterpret_cast<const float4*>(stF + q * kS + 4 * lane);
             const float4 f1 = *reinterpret_cast<const float4*>(stF + q * kS + 128 + 4 * lane);
             Fv[0] = f0.x; Fv[1] = f0.y; Fv[2] = f0.z; Fv[3] = f0.w;
@@ -328,37 +319,23 @@ __global__ void __launch_bounds__(dense::Cfg<ADJ>::THREADS, 1) dense_fb_kernel(c
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           z[j] = (t < n - 1) ? acc1[i][j] : 1.f;
-          if constexpr (ADJ) Bt[j] = (t < n - 1 && acc1[i][j] > 0.f) ? acc2[i][j] / acc1[i][j] : 0.f;
+          Bt[j] = (t < n - 1 && acc1[i][j] > 0.f) ? acc2[i][j] / acc1[i][j] : 0.f;
           zsum += z[j];
         }
         const float zinv = 1.f / warp_sum(zsum);
-        float gsum = 0.f, gc_ = 0.f;
+        float gsum = 0.f;
         float gm[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           z[j] *= zinv;
           gm[j] = x[j] * z[j];
           gsum += gm[j];
-          gc_ = fmaf(gm[j], cs[j], gc_);
         }
         const float den = warp_sum(gsum);
-        const float num = warp_sum(gc_);
         const float ginv = 1.f / den;
         const float wt = load_row(p.w, i, t);
-        if constexpr (!ADJ) {
-          if (act[i]) {
-            if (lane == 0) p.w_hat[static_cast<size_t>(qg[i]) * n + t] = num * ginv;
-            if (p.marginals) {
-              float* mr = p.marginals + (static_cast<size_t>(qg[i]) * n + t) * kS;
-              *reinterpret_cast<float4*>(mr + 4 * lane) =
-                  make_float4(gm[0] * ginv, gm[1] * ginv, gm[2] * ginv, gm[3] * ginv);
-              *reinterpret_cast<float4*>(mr + 128 + 4 * lane) =
-                  make_float4(gm[4] * ginv, gm[5] * ginv, gm[6] * ginv, gm[7] * ginv);
-            }
-          }
-        }
         float eps[8];
-        if constexpr (ADJ) {
+        {
           const float gt = load_row(p.g, i, t);
           const float wh = load_row(p.what_in, i, t);
           const float actf = act[i] ? 1.f : 0.f;
@@ -401,12 +378,12 @@ __global__ void __launch_bounds__(dense::Cfg<ADJ>::THREADS, 1) dense_fb_kernel(c
             const float v = ex2f(-(d * d) * sc2 - m2) * z[j];
             A1[a_index(st_of(lane, j), q)] = v;
             V8[j] = v;
-            if constexpr (ADJ) {
+            {
               W8[j] = v * (eps[j] + Bt[j]);
               A2[a_index(st_of(lane, j), q)] = W8[j];
             }
           }
-          if constexpr (ADJ) {
+          {
             if (p.ckv) {  // rows V = v_t, W = v_t (eps_t + B~_t) of the transition t-1 -> t
               float* vr = p.ckv + static_cast<size_t>(blockIdx.x) * p.ck_stride + (static_cast<size_t>(t - 1) * kM + q) * kS;
               float* wr = p.ckw + static_cast<size_t>(blockIdx.x) * p.ck_stride + (static_cast<size_t>(t - 1) * kM + q) * kS;
@@ -422,7 +399,7 @@ __global__ void __launch_bounds__(dense::Cfg<ADJ>::THREADS, 1) dense_fb_kernel(c
     }
   }
 
-  if constexpr (ADJ) {
+  {
     // Per-CTA codebook-gradient partial: sum the warps' per-lane accumulators in a fixed order.
     __syncthreads();
     float* red = Pc;  // [WARPS][S]
@@ -431,7 +408,7 @@ __global__ void __launch_bounds__(dense::Cfg<ADJ>::THREADS, 1) dense_fb_kernel(c
     __syncthreads();
     for (int s = tid; s < kS; s += NTH) {
       float v = 0.f;
-      for (int w = 0; w < Cfg<ADJ>::WARPS; ++w) v += red[w * kS + s];
+      for (int w = 0; w < Cfg::WARPS; ++w) v += red[w * kS + s];
       p.gc_part[static_cast<size_t>(blockIdx.x) * kS + s] = v;
     }
   }
@@ -440,41 +417,21 @@ __global__ void __launch_bounds__(dense::Cfg<ADJ>::THREADS, 1) dense_fb_kernel(c
 // ---------------------------------------------------------------------------
 // Host side.
 // ---------------------------------------------------------------------------
-size_t dense_smem_bytes(bool adjoint) {
+size_t dense_smem_bytes() {
   using namespace dense;
-  const size_t tiles = adjoint ? 2 : 1;
-  return sizeof(float) * (tiles * kS * kM + 2 * kKC * kS + tiles * kM * kS);
+  return sizeof(float) * (2 * kS * kM + 2 * kKC * kS + 2 * kM * kS);
 }
 
-cudaError_t dense_geometry(bool adjoint, int n_seq, int* grid) {
-  const void* fn = adjoint ? reinterpret_cast<const void*>(&dense_fb_kernel<true>)
-                           : reinterpret_cast<const void*>(&dense_fb_kernel<false>);
-  const size_t smem = dense_smem_bytes(adjoint);
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  int dev = 0, sms = 0, per_sm = 0;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  const int threads = adjoint ? dense::Cfg<true>::THREADS : dense::Cfg<false>::THREADS;
-  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem)) != cudaSuccess) return e;
-  if (per_sm < 1) return cudaErrorNotSupported;
-  const int blocks = (n_seq + dense::kM - 1) / dense::kM;
-  const int cap = per_sm * sms;
-  *grid = blocks < 1 ? 1 : (blocks < cap ? blocks : cap);
-  return cudaSuccess;
-}
-
-int dense_max_grid(bool adjoint) {
-  const void* fn = adjoint ? reinterpret_cast<const void*>(&dense_fb_kernel<true>)
-                           : reinterpret_cast<const void*>(&dense_fb_kernel<false>);
-  const size_t smem = dense_smem_bytes(adjoint);
-  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
+int dense_max_grid() {
+  const size_t smem = dense_smem_bytes();
+  if (cudaFuncSetAttribute(dense_adj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess)
     return 0;
   int dev = 0, sms = 0, per_sm = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  const int threads = adjoint ? dense::Cfg<true>::THREADS : dense::Cfg<false>::THREADS;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem) != cudaSuccess) return 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dense_adj_kernel, dense::Cfg::THREADS, smem) != cudaSuccess)
+    return 0;
   return per_sm * sms;
 }
 
@@ -484,15 +441,10 @@ cudaError_t launch_dense_prep(const float* lam, const DenseParams& p, cudaStream
   return cudaGetLastError();
 }
 
-cudaError_t launch_dense(const DenseParams& p, const float* lam, bool adjoint, int grid, cudaStream_t s, bool prep) {
+cudaError_t launch_dense(const DenseParams& p, const float* lam, int grid, cudaStream_t s, bool prep) {
   cudaError_t e = cudaSuccess;
   if (prep && (e = launch_dense_prep(lam, p, s)) != cudaSuccess) return e;
-  const size_t smem = dense_smem_bytes(adjoint);
-  if (adjoint) {
-    dense_fb_kernel<true><<<grid, dense::Cfg<true>::THREADS, smem, s>>>(p);
-  } else {
-    dense_fb_kernel<false><<<grid, dense::Cfg<false>::THREADS, smem, s>>>(p);
-  }
+  dense_adj_kernel<<<grid, dense::Cfg::THREADS, dense_smem_bytes(), s>>>(p);
   return cudaGetLastError();
 }
 

@@ -159,8 +159,9 @@ __global__ void dense_tc_mtab_kernel(const float* __restrict__ w, const float* _
   }
 }
 
+template <bool ADJ>
 __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::kThreads, 1)
-    dense_tc_fwd_kernel(const DenseTCParams p) {
+    dense_tc_kernel(const DenseTCParams p) {
   using namespace dtc;
   extern __shared__ __align__(16) unsigned char sm[];
   unsigned char* Bs = sm + kOffB;
@@ -184,7 +185,8 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
   const int row = (warp & 3) * 32 + (tid & 31);
   const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
   const int n = p.n, N = p.N;
-  const int ntiles = (N + kMR - 1) / kMR;
+  constexpr int kSeqs = ADJ ? kMR / 2 : kMR;  // sequences per tile
+  const int ntiles = (N + kSeqs - 1) / kSeqs;
   const float sc2 = p.sc2;
 
   if (warp == 0) {
@@ -366,6 +368,9 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
     tmem_wait_st();
   };
 
+  float gcacc[16];  // vector-Jacobian product: this thread's codebook-gradient sums
+#pragma unroll
+  for (int j = 0; j < 16; ++j) gcacc[j] = 0.f;
   float* ckbase = p.ck + static_cast<size_t>(cid * kCL + r) * p.ck_stride;      // [t][16 groups][128 rows] float4
   // [t][half][128 rows][2] partial sums, then [128 rows][half] the last forward row sums
   float* ptbase = p.part + static_cast<size_t>(cid * kCL + r) * p.part_stride;
@@ -374,6 +379,7 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
   };
 
   for (int tile = cid; tile < ntiles; tile += ncl) {
+    if constexpr (!ADJ) {
     const int q = tile * kMR + row;
     const bool act = q < N;
     const size_t qb = static_cast<size_t>(act ? q : 0) * n;  // padding rows run sequence 0 (discarded)
@@ -523,6 +529,216 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
       }
     }
     cluster_sync_all();  // partial sums read before the next tile rewrites them
+    } else {
+      // ------------- vector-Jacobian product: 64 sequences, two operands each -------------
+      // Row 2i + o of the MMA is operand o of sequence i of the tile: o = 0
+      // carries the vector (x forward, v backward), o = 1 the vector times
+      // its centred accumulator.  After a step the pair (2i, 2i + 1) trades
+      // halves so that each thread holds both sums for 16 states: thread o
+      // of the pair takes states c0 .. c0 + 15 of the CTA's block.
+      const int o = row & 1, qi = row >> 1;
+      const int ho = 2 * half + o;
+      const int c0 = 32 * half + 16 * o;
+      const int q = tile * kSeqs + qi;
+      const bool act = q < N;
+      const size_t qb = static_cast<size_t>(act ? q : 0) * n;  // padding sequences run sequence 0 (discarded)
+      float* ckx = p.ck + static_cast<size_t>(cid * kCL + r) * p.ck_stride;
+      float* ckf = p.ckf + static_cast<size_t>(cid * kCL + r) * p.ck_stride;
+      float* cks = p.cks + static_cast<size_t>(cid * kCL + r) * p.cks_stride;
+      // [t][pair half ho][float4 j][64 sequences] float4: a warp's stores are contiguous
+      auto ck_off = [&](int t, int j) { return ((static_cast<size_t>(t) * 4 + ho) * 4 + j) * (kSeqs * 4) + qi * 4; };
+      // per-row partial sums: [t][ho][64] for t < n, then [n][ho][64] last row sums, [n + 1][ho][64] D numerators
+      auto part_at = [&](float* base, int t) { return base + (static_cast<size_t>(t) * 4 + ho) * kSeqs + qi; };
+      // y (this thread's 32 sums of its row) -> a, b: the two operands' sums for states c0 .. c0 + 15
+      auto pair_split = [&](const float (&y)[32], float (&a)[16], float (&b)[16]) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float other = __shfl_xor_sync(0xffffffffu, o == 0 ? y[16 + j] : y[j], 1);
+          a[j] = o == 0 ? y[j] : other;
+          b[j] = o == 0 ? other : y[16 + j];
+        }
+      };
+      // the pair's operand rows from the two 16-state pieces of each thread
+      auto put_pair = [&](const float (&v1)[16], const float (&v2)[16]) {
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float other = __shfl_xor_sync(0xffffffffu, o == 0 ? v2[j] : v1[j], 1);
+          v[j] = o == 0 ? v1[j] : other;
+          v[16 + j] = o == 0 ? other : v2[j];
+        }
+        put_operand(v);
+      };
+      const float* cwq = cws + c0;
+
+      // ---------------- forward sweep: x_t and F~_t ----------------
+      if (n > 1) load_b(p.Bfwd);
+      cluster_arrive_relaxed();
+      if (!worker) issuer_sweep();
+      float wn = __ldg(p.w + qb), mn = __ldg(p.mtab + qb), gn = __ldg(p.g + qb), hn = __ldg(p.what_in + qb);
+      float xsum = 0.f, dnum = 0.f;  // over this thread's states: the vector and its D numerator
+      for (int t = 0; t < n && worker; ++t) {
+        float y[32], a[16], b[16];
+        float sprev = 1.f;
+        if (t > 0) {
+          const float s = step(t == 1, y);
+          sprev = __shfl_sync(0xffffffffu, s, (threadIdx.x & 31) & ~1);  // the pair's vector row sum
+          pair_split(y, a, b);
+          if (half == 0 && o == 0) cks[static_cast<size_t>(t - 1) * kSeqs + qi] = sprev;  // s_{t-1}
+        }
+        const float wt = wn, mt = mn, gt = gn, ht = hn;
+        if (t + 1 < n) {
+          wn = __ldg(p.w + qb + t + 1);
+          mn = __ldg(p.mtab + qb + t + 1);
+          gn = __ldg(p.g + qb + t + 1);
+          hn = __ldg(p.what_in + qb + t + 1);
+        }
+        const float inv = 1.f / sprev;
+        float x[16], f[16], x2[16];
+        xsum = 0.f;
+        dnum = 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float c = cwq[j];
+          const float d = wt - c;
+          const float e = ex2f(-(d * d) * sc2 - mt);
+          x[j] = (t > 0 ? a[j] * inv : 1.f) * e;
+          f[j] = (t > 0 && a[j] > 0.f) ? __fdividef(b[j], a[j]) : 0.f;
+          x2[j] = x[j] * (f[j] + gt * (c - ht));
+          xsum += x[j];
+          dnum += x2[j];
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          *reinterpret_cast<float4*>(ckx + ck_off(t, j)) = make_float4(x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3]);
+          *reinterpret_cast<float4*>(ckf + ck_off(t, j)) = make_float4(f[4 * j], f[4 * j + 1], f[4 * j + 2], f[4 * j + 3]);
+        }
+        if (t + 1 < n) put_pair(x, x2);
+      }
+      if (worker) {
+        *part_at(ptbase, n) = xsum;  // last vector's row sum, and D's numerator, over this thread's states
+        *part_at(ptbase, n + 1) = dnum;
+      }
+      cluster_wait_plain();
+      cluster_sync_all();  // every CTA's partial sums of the last step are written
+
+      // The last row sum s_{n-1} over all states (= den_{n-1}: z_{n-1} = 1) and
+      // D = sum_s gamma_{n-1}(s) (F~_{n-1}(s) + eps_{n-1}(s)), added in a fixed order.
+      float slast = 0.f, dsum = 0.f;
+#pragma unroll
+      for (int src = 0; src < kCL; ++src)
+#pragma unroll
+        for (int h4 = 0; h4 < 4; ++h4) {
+          const float* pb = p.part + static_cast<size_t>(cid * kCL + src) * p.part_stride;
+          slast += __ldcg(pb + (static_cast<size_t>(n) * 4 + h4) * kSeqs + qi);
+          dsum += __ldcg(pb + (static_cast<size_t>(n + 1) * 4 + h4) * kSeqs + qi);
+        }
+      const float Dv = dsum / slast;
+      if (worker && r == 0 && ho == 0 && act && !(isfinite(slast) && isfinite(Dv) && slast > 0.f))
+        atomicOr(p.status, kDevNonFinite);
+      // gamma's normaliser den_t = sum_s x_t(s) z_t(s) follows from the two
+      // recursions' row sums: den_{t-1} = den_t s_{t-1} / sigma_t (s: forward
+      // sums, sigma: backward sums), the same value on every CTA.
+      double den = static_cast<double>(slast);
+
+      // ---------------- backward sweep: z_t, B~_t, psi_t ----------------
+      if (n > 1) load_b(p.Bbwd);
+      cluster_arrive_relaxed();
+      if (!worker) issuer_sweep();
+      wn = __ldg(p.w + qb + n - 1);
+      mn = __ldg(p.mtab + qb + n - 1);
+      gn = __ldg(p.g + qb + n - 1);
+      hn = __ldg(p.what_in + qb + n - 1);
+      for (int t = n - 1; t >= 0 && worker; --t) {
+        float4 x4[4], f4[4];  // the stored forward values of the step, requested before the exchange
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          x4[j] = *reinterpret_cast<const float4*>(ckx + ck_off(t, j));
+          f4[j] = *reinterpret_cast<const float4*>(ckf + ck_off(t, j));
+        }
+        const float st = t < n - 1 ? cks[static_cast<size_t>(t) * kSeqs + qi] : 1.f;
+        float y[32], a[16], b[16];
+        float sig = 1.f;
+        if (t < n - 1) {
+          const float s = step(t == n - 2, y);
+          sig = __shfl_sync(0xffffffffu, s, (threadIdx.x & 31) & ~1);
+          pair_split(y, a, b);
+          den = den * static_cast<double>(st) / static_cast<double>(sig);
+        }
+        const float wt = wn, mt = mn, gt = gn, ht = hn;
+        if (t >= 1) {
+          wn = __ldg(p.w + qb + t - 1);
+          mn = __ldg(p.mtab + qb + t - 1);
+          gn = __ldg(p.g + qb + t - 1);
+          hn = __ldg(p.what_in + qb + t - 1);
+        }
+        const float inv = 1.f / sig;
+        const float rden = static_cast<float>(1.0 / den);
+        const float gsc = act ? gt : 0.f, tsc = act ? p.two_over_T : 0.f;
+        float gw = 0.f;
+        float v1[16], v2[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float xs = (j & 3) == 0 ? x4[j >> 2].x : (j & 3) == 1 ? x4[j >> 2].y : (j & 3) == 2 ? x4[j >> 2].z : x4[j >> 2].w;
+          const float fs = (j & 3) == 0 ? f4[j >> 2].x : (j & 3) == 1 ? f4[j >> 2].y : (j & 3) == 2 ? f4[j >> 2].z : f4[j >> 2].w;
+          const float c = cwq[j];
+          const float z = t < n - 1 ? a[j] * inv : 1.f;
+          const float bt = (t < n - 1 && a[j] > 0.f) ? __fdividef(b[j], a[j]) : 0.f;
+          const float eps = gt * (c - ht);
+          const float gam = xs * z * rden;
+          const float psi = gam * (fs + eps + bt - Dv);
+          gw = fmaf(psi, c, gw);
+          gcacc[j] += fmaf(gsc, gam, tsc * psi * (wt - c));
+          const float d = wt - c;
+          v1[j] = ex2f(-(d * d) * sc2 - mt) * z;
+          v2[j] = v1[j] * (eps + bt);
+        }
+        *part_at(ptbase, t) = gw;
+        if (t >= 1) put_pair(v1, v2);
+      }
+      cluster_wait_plain();
+      cluster_sync_all();  // every CTA's partial sums are written
+
+      // grad_w: CTA r takes the steps t = r, r + 4, ...; the partial sums over
+      // 4 CTAs x 4 pieces of 16 states are added in a fixed order.
+      for (int t = r + kCL * (tid >> 6); t < n && worker; t += 4 * kCL) {
+        const int qq = tid & (kSeqs - 1);
+        const int qg = tile * kSeqs + qq;
+        if (qg >= N) continue;
+        float gw = 0.f;
+#pragma unroll
+        for (int src = 0; src < kCL; ++src)
+#pragma unroll
+          for (int h4 = 0; h4 < 4; ++h4)
+            gw += __ldcg(p.part + static_cast<size_t>(cid * kCL + src) * p.part_stride +
+                         (static_cast<size_t>(t) * 4 + h4) * kSeqs + qq);
+        p.grad_w[static_cast<size_t>(qg) * n + t] = p.two_over_T * gw;
+      }
+      cluster_sync_all();  // partial sums read before the next tile rewrites them
+    }
+  }
+
+  if constexpr (ADJ) {
+    // This CTA's 64 codebook-gradient sums: over the 16 sequences of a warp
+    // with equal pair side (lane shuffles), then over the 4 lane quadrants
+    // (the receive area is free now), in a fixed order.
+    float* red = reinterpret_cast<float*>(Rx);  // [4 quadrants][64 states]
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      float v = gcacc[j];
+#pragma unroll
+      for (int off = 2; off < 32; off <<= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+      gcacc[j] = v;
+    }
+    if (worker && (tid & 31) < 2) {
+      const int c0 = 32 * half + 16 * (tid & 1);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) red[(warp & 3) * kSlice + c0 + j] = gcacc[j];
+    }
+    __syncthreads();
+    if (tid < kSlice)
+      p.gc_part[static_cast<size_t>(cid) * kS + r * kSlice + tid] =
+          ((red[tid] + red[kSlice + tid]) + red[2 * kSlice + tid]) + red[3 * kSlice + tid];
   }
 
   tc_fence_before();
@@ -540,19 +756,20 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
 size_t dense_tc_smem_bytes() { return dtc::kSmemBytes; }
 
 namespace {
-// Per device: the kernel's shared-memory attribute is set and its cluster
-// occupancy queried once, so that later calls issue no driver queries (a
-// query can wait behind other users of the driver).  0 = not yet known.
+// Per device and variant: the kernel's shared-memory attribute is set and its
+// cluster occupancy queried once, so that later calls issue no driver queries
+// (a query can wait behind other users of the driver).  0 = not yet known.
 constexpr int kMaxDevices = 64;
-int g_tc_clusters[kMaxDevices] = {};
+int g_tc_clusters[2][kMaxDevices] = {};
 
+template <bool ADJ>
 int tc_clusters_of_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
-  if (dev < kMaxDevices && g_tc_clusters[dev] > 0) return g_tc_clusters[dev];
+  if (dev < kMaxDevices && g_tc_clusters[ADJ][dev] > 0) return g_tc_clusters[ADJ][dev];
   const size_t smem = dense_tc_smem_bytes();
-  if (cudaFuncSetAttribute(dense_tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-      cudaSuccess)
+  if (cudaFuncSetAttribute(dense_tc_kernel<ADJ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
     return 0;
   int sms = 0;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
@@ -561,15 +778,17 @@ int tc_clusters_of_device() {
   cfg.blockDim = dim3(dtc::kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   int clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&clusters, dense_tc_fwd_kernel, &cfg) != cudaSuccess) return 0;
-  if (dev < kMaxDevices) g_tc_clusters[dev] = clusters;
+  if (cudaOccupancyMaxActiveClusters(&clusters, dense_tc_kernel<ADJ>, &cfg) != cudaSuccess) return 0;
+  if (dev < kMaxDevices) g_tc_clusters[ADJ][dev] = clusters;
   return clusters;
 }
 }  // namespace
 
-int dense_tc_max_clusters() { return tc_clusters_of_device(); }
+int dense_tc_max_clusters(bool adjoint) {
+  return adjoint ? tc_clusters_of_device<true>() : tc_clusters_of_device<false>();
+}
 
-cudaError_t launch_dense_tc_forward(const DenseTCParams& p, const float* lam, int clusters, cudaStream_t s) {
+cudaError_t launch_dense_tc(const DenseTCParams& p, const float* lam, bool adjoint, int clusters, cudaStream_t s) {
   using namespace dtc;
   dense_tc_prep_kernel<<<(kS * kS + 255) / 256, 256, 0, s>>>(lam, p.Bfwd, p.Bbwd);
   cudaError_t e = cudaGetLastError();
@@ -579,8 +798,12 @@ cudaError_t launch_dense_tc_forward(const DenseTCParams& p, const float* lam, in
   dense_tc_mtab_kernel<<<static_cast<unsigned>(blocks < 4096 ? blocks : 4096), kS, 0, s>>>(p.w, p.codebook, p.sc2, total,
                                                                                          p.mtab);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (tc_clusters_of_device() < 1) return cudaErrorNotSupported;  // also sets the shared-memory attribute
-  dense_tc_fwd_kernel<<<clusters * kCL, kThreads, dense_tc_smem_bytes(), s>>>(p);
+  if (dense_tc_max_clusters(adjoint) < 1) return cudaErrorNotSupported;  // also sets the shared-memory attribute
+  if (adjoint) {
+    dense_tc_kernel<true><<<clusters * kCL, kThreads, dense_tc_smem_bytes(), s>>>(p);
+  } else {
+    dense_tc_kernel<false><<<clusters * kCL, kThreads, dense_tc_smem_bytes(), s>>>(p);
+  }
   return cudaGetLastError();
 }
 

@@ -43,10 +43,14 @@ def test_log_transition_gradient_parity(B, n, N, T):
     gw, gc, gl = B.bcjr_dense_backward(dg, dw, dc, dl, w_hat, T, want_grad_log_trans=True)
     gw0, gc0 = B.bcjr_dense_backward(dg, dw, dc, dl, w_hat, T)
     torch.cuda.synchronize()
-    # the extra outputs change nothing in the others
-    assert torch.equal(gw, gw0)
-    assert torch.equal(gc, gc0)
+    # The extra output leaves the others unchanged up to float32 rounding: the
+    # plain call runs the tensor-core adjoint, this one the kernel that also
+    # writes the rows of the log-transition gradient.
+    assert_rel_l2(gw, to_np(gw0), 1e-5, "grad_w of the two calls")
+    assert_rel_l2(gc, to_np(gc0), 1e-5, "grad_codebook of the two calls")
     o_gw, o_gc, o_gl = oracle.dense_backward(g, w, c, lam, T, want_grad_lam=True)
+    assert_rel_l2(gw0, o_gw, GRAD_REL_L2, "grad_w (plain call)")
+    assert_rel_l2(gc0, o_gc, GRAD_REL_L2, "grad_codebook (plain call)")
     if n == 1:
         assert bool((gl == 0).all())
         return
@@ -123,14 +127,16 @@ def test_dense_autograd_function(B):
     lv2 = lam.cuda()
     w2 = w.cuda().requires_grad_(True)
     (B.dense_soft_quantize(w2, c.cuda(), lv2, T) * g.cuda()).sum().backward()
-    assert torch.equal(w2.grad, wv.grad)
+    assert_rel_l2(w2.grad, o_gw, GRAD_REL_L2, "grad_w (plain call)")
+    assert_rel_l2(w2.grad, to_np(wv.grad), 1e-5, "grad_w of the two calls")
 
 
 @pytest.mark.slow
 def test_log_transition_gradient_full_workload(B):
     # 4096 sequences x 4096 steps (the dense workload): the oracle cannot run
     # at this size, so check what holds at any size -- the zero sum, agreement
-    # of the other outputs with the plain backward call, run-to-run identity.
+    # of the other outputs with the plain backward call (a different kernel:
+    # float32-level agreement), run-to-run identity.
     W = I.WORKLOADS["dense_S256"]
     n, N, T = W["seq_len"], W["n_seq"], W["T"][0]
     c, w, g, lam = I.codebook(S).cuda(), I.weights(N, n).cuda(), I.upstream_grad(N, n).cuda(), I.log_transition(S).cuda()
@@ -139,7 +145,8 @@ def test_log_transition_gradient_full_workload(B):
     gw0, gc0 = B.bcjr_dense_backward(g, w, c, lam, w_hat, T)
     _, _, gl2 = B.bcjr_dense_backward(g, w, c, lam, w_hat, T, want_grad_log_trans=True)
     torch.cuda.synchronize()
-    assert torch.equal(gw, gw0) and torch.equal(gc, gc0)
+    assert_rel_l2(gw, to_np(gw0), 1e-5, "grad_w of the two calls")
+    assert_rel_l2(gc, to_np(gc0), 1e-5, "grad_codebook of the two calls")
     assert torch.equal(gl, gl2)
     x = gl.double()
     assert bool(torch.isfinite(x).all())
