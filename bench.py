@@ -408,9 +408,12 @@ def run_gpu(args):
             try:
                 cores = len(os.sched_getaffinity(0))
                 sample = max(1, min(cores, 16))
-                rate, threads, dt = oracle_sample_rate(sample, [temps[0]])
+                # the first, a middle and the last temperature of the sweep (about 15 s on 16 cores)
+                ts = [temps[0], temps[len(temps) // 2], temps[-1]]
+                rate, threads, dt = oracle_sample_rate(sample, ts)
                 line["cpu_baseline"] = {"value": rate, "unit": "weights/s", "cores": threads, "kind": "oracle",
-                                        "sample": f"{sample} whole sequences (fwd+bwd at T={temps[0]}), "
+                                        "sample": f"{sample} whole sequences of the workload, fwd+bwd at each of "
+                                                  f"T = {', '.join(f'{t:.4g}' for t in ts)}, "
                                                   f"{dt:.1f} s of CPU work"}
             except Exception as e:  # pragma: no cover
                 line["cpu_baseline"] = {"value": None, "error": str(e)}
