@@ -171,8 +171,9 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
   uint64_t* bar_c = reinterpret_cast<uint64_t*>(sm + kOffBar);  // [4] output blocks committed, in issue order
   uint64_t* bar_rx = bar_c + 4;                                  // [3] a receive slot filled
   uint64_t* bar_b = bar_c + 7;                                   // resident slice loaded
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_c + 8);
-  int* abort_flag = reinterpret_cast<int*>(bar_c + 9);
+  uint64_t* bar_sum = bar_c + 8;                                 // row-sum MMAs done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_c + 9);
+  int* abort_flag = reinterpret_cast<int*>(bar_c + 10);
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int r = static_cast<int>(cluster_rank());
@@ -196,7 +197,7 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   if (tid == 0) {
-    for (int i = 0; i < 8; ++i) mbar_init(bar_c + i, 1);
+    for (int i = 0; i < 9; ++i) mbar_init(bar_c + i, 1);
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -212,7 +213,7 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
     for (int i = 0; i < kCL - 1; ++i) mbar_arm(bar_rx + i, kRxSlot);
   cluster_sync_all();  // every CTA's barriers are initialised (and armed) before any remote store
 
-  uint32_t ph_c[4] = {0, 0, 0, 0}, ph_b = 0;
+  uint32_t ph_c[4] = {0, 0, 0, 0}, ph_b = 0, ph_sum = 0;
   uint32_t ph_rx = 0;  // parity of receive slot s in bit s
   // After one wait of this CTA gave up, no thread waits again (the call's results are void).
   auto waitb = [&](uint64_t* bar, uint32_t& ph) {
@@ -233,9 +234,10 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
   };
   // Output block of issue slot k: the other CTAs' blocks first, the own one last.
   auto block_of = [&](int k) { return (r + 1 + k) & (kCL - 1); };
-  // The MMAs of one step (tid 0), one commit per output block; the operand's
-  // row sums over this CTA's states (head and tail times a tile of ones) go
-  // with the first block.
+  // The MMAs of one step (one thread), one commit per output block; the
+  // operand's row sums over this CTA's states (head and tail times a tile of
+  // ones) follow the first block, so that the exchange starts as early as it
+  // can.
   auto issue_mma = [&](bool first_of_sweep) {
     if (first_of_sweep) waitb(bar_b, ph_b);
     tc_fence_after();
@@ -246,14 +248,6 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
       const int blk = block_of(k);
       const uint32_t d = tmem + static_cast<uint32_t>(blk * kSlice);
       if (go) {
-        if (k == 0) {
-          const uint64_t od = smem_desc(smem_u32(ones));
-#pragma unroll
-          for (int c = 0; c < kKC; ++c) {
-            mma_tf32_ts(tmem + kTSum, tmem + kTAh + 8 * c, od, kIdescN16, c > 0 ? 1u : 0u);
-            mma_tf32_ts(tmem + kTSum, tmem + kTAl + 8 * c, od, kIdescN16, 1u);
-          }
-        }
 #pragma unroll
         for (int c = 0; c < kKC; ++c) {
           const uint32_t bh = b0 + (2 * c) * kBTile + blk * kBBlock, bl = bh + kBTile;
@@ -264,13 +258,24 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
         }
       }
       mma_commit(bar_c + k);
+      if (k == 0) {
+        if (go) {
+          const uint64_t od = smem_desc(smem_u32(ones));
+#pragma unroll
+          for (int c = 0; c < kKC; ++c) {
+            mma_tf32_ts(tmem + kTSum, tmem + kTAh + 8 * c, od, kIdescN16, c > 0 ? 1u : 0u);
+            mma_tf32_ts(tmem + kTSum, tmem + kTAl + 8 * c, od, kIdescN16, 1u);
+          }
+        }
+        mma_commit(bar_sum);
+      }
     }
   };
   // One step's contraction and reduce-scatter.  Every thread sends its half of
   // the other CTAs' blocks of its row as they complete (st.async into the
   // receiver's slot: 16 groups x 128 rows of float4, so a warp's stores are
-  // contiguous; half 0 adds the row sum), then adds the three received halves
-  // to its own into y.  Returns the row's sum of the consumed vector over all
+  // contiguous; after the first block, half 0 sends the row sum to all three),
+  // then adds the three received halves to its own into y.  Returns the row's sum of the consumed vector over all
   // 256 states, added in CTA order so that every CTA gets the same value.
   auto step = [&](bool first_of_sweep, float (&y)[32]) -> float {
     tc_fence_before();
@@ -284,14 +289,7 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
       tc_fence_after();
       uint32_t v[32];
       tmem_ld32_async(tmem + lane_off + static_cast<uint32_t>(blk * kSlice + 32 * half), v);
-      if (k == 0) {
-        uint32_t s1;
-        asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(s1) : "r"(tmem + lane_off + kTSum));
-        tmem_wait_ld();
-        rs = __uint_as_float(s1);
-      } else {
-        tmem_wait_ld();
-      }
+      tmem_wait_ld();
       const uint32_t slot = static_cast<uint32_t>(r < blk ? r : r - 1);
       const uint32_t dst = mapa_u32(smem_u32(Rx) + slot * kRxSlot, static_cast<uint32_t>(blk));
       const uint32_t rbar = mapa_u32(smem_u32(bar_rx + slot), static_cast<uint32_t>(blk));
@@ -300,7 +298,24 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
         st_async_v4f32(dst + static_cast<uint32_t>(((8 * half + g) * kMR + row) * 16), __uint_as_float(v[4 * g]),
                        __uint_as_float(v[4 * g + 1]), __uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3]),
                        rbar);
-      if (half == 0) st_async_f32(dst + kRxData + static_cast<uint32_t>(row * 4), rs, rbar);
+      if (k == 0) {
+        waitb(bar_sum, ph_sum);
+        tc_fence_after();
+        uint32_t s1;
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(s1) : "r"(tmem + lane_off + kTSum));
+        tmem_wait_ld();
+        rs = __uint_as_float(s1);
+        if (half == 0) {
+#pragma unroll
+          for (int j = 1; j < kCL; ++j) {
+            const int b2 = (r + j) & (kCL - 1);
+            const uint32_t sl2 = static_cast<uint32_t>(r < b2 ? r : r - 1);
+            st_async_f32(mapa_u32(smem_u32(Rx) + sl2 * kRxSlot + kRxData + static_cast<uint32_t>(row * 4),
+                                  static_cast<uint32_t>(b2)),
+                         rs, mapa_u32(smem_u32(bar_rx + sl2), static_cast<uint32_t>(b2)));
+          }
+        }
+      }
     }
     // Received halves: added as they land, in the order the senders finish
     // them (CTA r - 1 computes this CTA's block first); the own block's
