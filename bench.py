@@ -624,9 +624,10 @@ def run_dense(args):
                                                        N, W["n_seq"])},
             "kernels_ms": {"bcjr_dense_forward": 1e3 * fwd_s,
                            ("bcjr_dense_backward_lambda" if wl else "bcjr_dense_backward"): 1e3 * bwd_s},
-            # forward: prep, reference, kernel; backward: prep, reference, kernel, codebook reduction
-            # (with dL/dLambda: prep, adjoint, codebook reduction, row-product sum, reduction)
-            "gpu_launches": (3 + (5 if wl else 4)) * args.steps,
+            # forward: prep, reference, kernel; backward: prep, reference, kernel, codebook reduction;
+            # with dL/dLambda the backward call runs those and the row-product sum and its reduction
+            # once per chunk of one 64-sequence tile per cluster (33 clusters fit on a B200)
+            "gpu_launches": (3 + (6 * -(-N // (64 * 33)) if wl else 4)) * args.steps,
             "clocks": clocks,
         }
         if wl:

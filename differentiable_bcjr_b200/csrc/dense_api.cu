@@ -14,59 +14,26 @@ constexpr size_t kAlign = 256;
 
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 
-struct DenseLayout {
-  size_t P, PT, ckx, ckf, ckv, ckw, mtab, gc, dlpart, total, ck_stride, mt_stride;
-};
-
-// Workspace of the vector-Jacobian product with the log-transition gradient:
-// P and P^T, per CTA the rows X, U, V, W of that gradient (X and U in the
-// places of the stored forward values) and the step references, the codebook
-// partials, and `dl_parts` [S][S] partial sums of the row products.
-DenseLayout dense_layout(int grid, int n, int dl_parts) {
-  const size_t S = bcjr::kDenseStates, M = bcjr::kDenseRows;
-  DenseLayout l = {};
-  l.ck_stride = static_cast<size_t>(n) * M * S;
-  l.mt_stride = static_cast<size_t>(n) * M;
-  const size_t ck_bytes = static_cast<size_t>(grid) * l.ck_stride * sizeof(float);
-  size_t off = kHeader;
-  l.P = off;
-  off = align_up(off + S * S * sizeof(float));
-  l.PT = off;
-  off = align_up(off + S * S * sizeof(float));
-  l.ckx = off;
-  off = align_up(off + ck_bytes);
-  l.ckf = off;
-  off = align_up(off + ck_bytes);
-  l.ckv = off;
-  off = align_up(off + ck_bytes);
-  l.ckw = off;
-  off = align_up(off + ck_bytes);
-  l.mtab = off;
-  off = align_up(off + static_cast<size_t>(grid) * l.mt_stride * sizeof(float));
-  l.gc = off;
-  off = align_up(off + static_cast<size_t>(grid) * S * sizeof(float));
-  l.dlpart = off;
-  off = align_up(off + static_cast<size_t>(dl_parts) * S * S * sizeof(float));
-  l.total = off;
-  return l;
-}
-
 // Workspace of the tensor-core calls: the transfer matrix as two sets of
 // resident operand slices, the emission reference of every step, and per CTA
 // of the resident clusters its stored forward values and partial sums (the
 // adjoint adds the F~ ratios, the forward row sums and the codebook-gradient
-// partials of each cluster).
+// partials of each cluster).  With the log-transition gradient it adds P
+// row-major, the rows X, U, V, W of every cluster's tile and `dl_parts`
+// [S][S] partial sums of their products.
 struct DenseTCLayout {
-  size_t Bfwd, Bbwd, mtab, ck, ckf, cks, part, gc, total, ck_stride, cks_stride, part_stride;
+  size_t Bfwd, Bbwd, mtab, ck, ckf, cks, part, gc, P, rows, dlpart, total;
+  size_t ck_stride, cks_stride, part_stride, row_region;
 };
 
-DenseTCLayout dense_tc_layout(bool adjoint, int clusters, int n, int N) {
+DenseTCLayout dense_tc_layout(bool adjoint, int clusters, int n, int N, int dl_parts) {
   const size_t S = bcjr::kDenseStates, CL = bcjr::kDenseTCCluster;
   const size_t seqs = static_cast<size_t>(bcjr::dense_tc_tile_seqs(adjoint));
   DenseTCLayout l = {};
   l.ck_stride = static_cast<size_t>(n) * seqs * (S / CL);
   l.cks_stride = adjoint ? static_cast<size_t>(n) * seqs : 0;
   l.part_stride = adjoint ? static_cast<size_t>(n + 2) * 4 * seqs : static_cast<size_t>(2 * n + 1) * seqs * 2;
+  l.row_region = dl_parts > 0 ? static_cast<size_t>(n - 1) * seqs * S : 0;
   const size_t ctas = static_cast<size_t>(clusters) * CL;
   size_t off = kHeader;
   l.Bfwd = off;
@@ -85,10 +52,17 @@ DenseTCLayout dense_tc_layout(bool adjoint, int clusters, int n, int N) {
   off = align_up(off + ctas * l.part_stride * sizeof(float));
   l.gc = off;
   if (adjoint) off = align_up(off + static_cast<size_t>(clusters) * S * sizeof(float));
+  l.P = off;
+  if (dl_parts > 0) off = align_up(off + S * S * sizeof(float));
+  l.rows = off;
+  off = align_up(off + 4 * static_cast<size_t>(clusters) * l.row_region * sizeof(float));
+  l.dlpart = off;
+  off = align_up(off + static_cast<size_t>(dl_parts) * S * S * sizeof(float));
   l.total = off;
   return l;
 }
 
+// Clusters of one launch: one per tile, at most as many as fit.
 bcjr_status dense_tc_clusters(bool adjoint, int N, int* clusters) {
   const int cap = bcjr::dense_tc_max_clusters(adjoint);
   if (cap < 1) return BCJR_ERR_UNSUPPORTED;
@@ -98,21 +72,11 @@ bcjr_status dense_tc_clusters(bool adjoint, int N, int* clusters) {
   return BCJR_OK;
 }
 
-// Launch geometry of the backward call that also returns the log-transition
-// gradient: the rows of that gradient live in per-CTA regions, so every CTA
-// takes one block of 32 sequences per launch and longer batches run in chunks
-// of 32 x (CTAs that fit) sequences.  `parts` = partial sums of the reduction
-// (one per SM).
-bcjr_status dlam_geometry(int N, int* grid, int* chunk, int* parts) {
-  const int cap = bcjr::dense_max_grid();
-  if (cap < 1) return BCJR_ERR_UNSUPPORTED;
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+// Partial sums of the log-transition gradient's row-product sum: one per SM.
+bcjr_status dlam_parts(int* parts) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(parts, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return BCJR_ERR_CUDA;
-  const int blocks = (N + bcjr::kDenseRows - 1) / bcjr::kDenseRows;
-  *grid = blocks < 1 ? 1 : (blocks < cap ? blocks : cap);
-  *chunk = cap * bcjr::kDenseRows;
-  *parts = sms;
   return BCJR_OK;
 }
 
@@ -157,108 +121,88 @@ bcjr_status dense_common(bool adjoint, const float* g, const float* w, const flo
     if (marginals && !aligned(marginals, 16)) return BCJR_ERR_INVALID_ARG;
   }
   if (!ws || !aligned(ws, kAlign)) return BCJR_ERR_WORKSPACE;
-  if (!grad_lam) {
-    // The soft codeword and the plain vector-Jacobian product: the tensor-core
-    // kernels (dense_tc_kernel.cu).
-    int clusters = 0;
-    if ((st = dense_tc_clusters(adjoint, N, &clusters)) != BCJR_OK) return st;
-    const DenseTCLayout lt = dense_tc_layout(adjoint, clusters, n, N);
-    if (ws_bytes < lt.total) return BCJR_ERR_WORKSPACE;
-    char* b = static_cast<char*>(ws);
-    bcjr::DenseTCParams tp = {};
-    tp.w = w;
-    tp.codebook = c;
-    tp.g = g;
-    tp.what_in = what_in;
-    tp.mtab = reinterpret_cast<float*>(b + lt.mtab);
-    tp.Bfwd = reinterpret_cast<float*>(b + lt.Bfwd);
-    tp.Bbwd = reinterpret_cast<float*>(b + lt.Bbwd);
-    tp.ck = reinterpret_cast<float*>(b + lt.ck);
-    tp.ckf = reinterpret_cast<float*>(b + lt.ckf);
-    tp.cks = reinterpret_cast<float*>(b + lt.cks);
-    tp.part = reinterpret_cast<float*>(b + lt.part);
-    tp.gc_part = reinterpret_cast<float*>(b + lt.gc);
-    tp.w_hat = w_hat;
-    tp.marginals = marginals;
-    tp.log_z = log_z;
-    tp.grad_w = grad_w;
-    tp.status = reinterpret_cast<int*>(b);
-    tp.ck_stride = lt.ck_stride;
-    tp.cks_stride = lt.cks_stride;
-    tp.part_stride = lt.part_stride;
-    tp.sc2 = static_cast<float>(1.4426950408889634 / static_cast<double>(T));
-    tp.two_over_T = static_cast<float>(2.0 / static_cast<double>(T));
-    tp.n = n;
-    tp.N = N;
-    if ((st = from_cuda(cudaMemsetAsync(ws, 0, sizeof(int), s))) != BCJR_OK) return st;
+  // All three calls run the tensor-core kernels (dense_tc_kernel.cu).  With
+  // the log-transition gradient the adjoint runs in chunks of one tile per
+  // cluster, writing the rows X, U, V, W of each chunk's transitions, which the
+  // tensor-core row-product sum (dense_dlam_kernel.cu) adds up after each chunk.
+  const bool dl = grad_lam != nullptr;
+  int clusters = 0, parts = 0;
+  if ((st = dense_tc_clusters(adjoint, N, &clusters)) != BCJR_OK) return st;
+  if (dl && (st = dlam_parts(&parts)) != BCJR_OK) return st;
+  const int per = bcjr::dense_tc_tile_seqs(adjoint);
+  const int chunk = dl ? clusters * per : N;
+  const DenseTCLayout lt = dense_tc_layout(adjoint, clusters, n, chunk < N ? chunk : N, dl ? parts : 0);
+  if (ws_bytes < lt.total) return BCJR_ERR_WORKSPACE;
+  char* b = static_cast<char*>(ws);
+  bcjr::DenseTCParams tp = {};
+  tp.w = w;
+  tp.codebook = c;
+  tp.g = g;
+  tp.what_in = what_in;
+  tp.mtab = reinterpret_cast<float*>(b + lt.mtab);
+  tp.Bfwd = reinterpret_cast<float*>(b + lt.Bfwd);
+  tp.Bbwd = reinterpret_cast<float*>(b + lt.Bbwd);
+  tp.ck = reinterpret_cast<float*>(b + lt.ck);
+  tp.ckf = reinterpret_cast<float*>(b + lt.ckf);
+  tp.cks = reinterpret_cast<float*>(b + lt.cks);
+  tp.part = reinterpret_cast<float*>(b + lt.part);
+  tp.gc_part = reinterpret_cast<float*>(b + lt.gc);
+  tp.w_hat = w_hat;
+  tp.marginals = marginals;
+  tp.log_z = log_z;
+  tp.grad_w = grad_w;
+  tp.status = reinterpret_cast<int*>(b);
+  tp.ck_stride = lt.ck_stride;
+  tp.cks_stride = lt.cks_stride;
+  tp.part_stride = lt.part_stride;
+  tp.sc2 = static_cast<float>(1.4426950408889634 / static_cast<double>(T));
+  tp.two_over_T = static_cast<float>(2.0 / static_cast<double>(T));
+  tp.n = n;
+  tp.N = N;
+  if ((st = from_cuda(cudaMemsetAsync(ws, 0, sizeof(int), s))) != BCJR_OK) return st;
+  if (!dl) {
     if ((st = from_cuda(bcjr::launch_dense_tc(tp, lam, adjoint, clusters, s))) != BCJR_OK) return st;
     if (adjoint) return from_cuda(bcjr::launch_gradc_reduce(tp.gc_part, clusters, S, grad_c, accumulate, s));
     return BCJR_OK;
   }
-  // The vector-Jacobian product with the log-transition gradient (SIMT kernel
-  // writing full-width rows for the tensor-core row-product sum).
-  int grid = 0, chunk = N, parts = 0;
-  if ((st = dlam_geometry(N, &grid, &chunk, &parts)) != BCJR_OK) return st;
-  const DenseLayout lay = dense_layout(grid, n, parts);
-  if (ws_bytes < lay.total) return BCJR_ERR_WORKSPACE;
-  char* base = static_cast<char*>(ws);
-  bcjr::DenseParams p = {};
-  p.w = w;
-  p.codebook = c;
-  p.g = g;
-  p.what_in = what_in;
-  p.w_hat = w_hat;
-  p.marginals = marginals;
-  p.log_z = log_z;
-  p.grad_w = grad_w;
-  p.gc_part = reinterpret_cast<float*>(base + lay.gc);
-  p.P = reinterpret_cast<const float*>(base + lay.P);
-  p.PT = reinterpret_cast<const float*>(base + lay.PT);
-  p.ckx = reinterpret_cast<float*>(base + lay.ckx);
-  p.ckf = reinterpret_cast<float*>(base + lay.ckf);
-  p.ckv = reinterpret_cast<float*>(base + lay.ckv);
-  p.ckw = reinterpret_cast<float*>(base + lay.ckw);
-  p.mtab = reinterpret_cast<float*>(base + lay.mtab);
-  p.status = reinterpret_cast<int*>(base);
-  p.ck_stride = lay.ck_stride;
-  p.mt_stride = lay.mt_stride;
-  p.sc2 = static_cast<float>(1.4426950408889634 / static_cast<double>(T));
-  p.two_over_T = static_cast<float>(2.0 / static_cast<double>(T));
-  p.n = n;
-  p.N = N;
-  if ((st = from_cuda(cudaMemsetAsync(ws, 0, sizeof(int), s))) != BCJR_OK) return st;
-  // Backward call with the log-transition gradient, chunk by chunk: each
-  // chunk's backward kernel writes the rows X, U, V, W of its transitions, the
-  // tensor-core kernel sums them into per-SM partials, and the reductions add
-  // the chunk's codebook and log-transition gradients to the outputs.
-  float* dlpart = reinterpret_cast<float*>(base + lay.dlpart);
+  float* rows = reinterpret_cast<float*>(b + lt.rows);
+  const size_t rstride = static_cast<size_t>(clusters) * lt.row_region;
+  if (n > 1) {
+    tp.P = reinterpret_cast<float*>(b + lt.P);
+    tp.rowX = rows;
+    tp.rowU = rows + rstride;
+    tp.rowV = rows + 2 * rstride;
+    tp.rowW = rows + 3 * rstride;
+    tp.row_region = lt.row_region;
+  }
+  float* dlpart = reinterpret_cast<float*>(b + lt.dlpart);
   for (int c0 = 0; c0 < N; c0 += chunk) {
     const int Nc = (N - c0) < chunk ? (N - c0) : chunk;
     const int acc = (accumulate || c0 > 0) ? 1 : 0;
     const size_t off = static_cast<size_t>(c0) * n;
-    bcjr::DenseParams pc = p;
+    bcjr::DenseTCParams pc = tp;
     pc.w = w + off;
     pc.g = g + off;
     pc.what_in = what_in + off;
     pc.grad_w = grad_w + off;
     pc.N = Nc;
-    const int grid_c = (Nc + bcjr::kDenseRows - 1) / bcjr::kDenseRows;
-    if ((st = from_cuda(bcjr::launch_dense(pc, lam, grid_c, s, c0 == 0))) != BCJR_OK) return st;
-    if ((st = from_cuda(bcjr::launch_gradc_reduce(pc.gc_part, grid_c, S, grad_c, acc, s))) != BCJR_OK) return st;
+    const int cl_c = (Nc + per - 1) / per;
+    if ((st = from_cuda(bcjr::launch_dense_tc(pc, lam, true, cl_c, s))) != BCJR_OK) return st;
+    if ((st = from_cuda(bcjr::launch_gradc_reduce(pc.gc_part, cl_c, S, grad_c, acc, s))) != BCJR_OK) return st;
     if (n == 1) {  // no transitions: the gradient is zero
       if (!acc && (st = from_cuda(cudaMemsetAsync(grad_lam, 0, S * S * sizeof(float), s))) != BCJR_OK) return st;
       continue;
     }
     bcjr::DlamParams dp = {};
-    dp.X = pc.ckx;
-    dp.U = pc.ckf;
-    dp.V = pc.ckv;
-    dp.W = pc.ckw;
+    dp.X = pc.rowX;
+    dp.U = pc.rowU;
+    dp.V = pc.rowV;
+    dp.W = pc.rowW;
     dp.part = dlpart;
     dp.status = pc.status;
-    dp.region_stride = static_cast<long long>(lay.ck_stride);
-    dp.spr = static_cast<long long>(n - 1) * (bcjr::kDenseRows / 8);
-    dp.total_stages = static_cast<long long>(grid_c) * dp.spr;
+    dp.region_stride = static_cast<long long>(lt.row_region);
+    dp.spr = static_cast<long long>(n - 1) * (per / 8);
+    dp.total_stages = static_cast<long long>(cl_c) * dp.spr;
     int gd = 0;
     if ((st = from_cuda(bcjr::dlam_grid(dp.total_stages, &gd))) != BCJR_OK) return st;
     if (gd > parts) gd = parts;
@@ -274,15 +218,13 @@ size_t bcjr_dense_workspace_size_impl(int op, int n_states, int seq_len, int n_s
   if (n_states != bcjr::kDenseStates || seq_len < 1 || n_seq < 0) return 0;
   if (check_options(opt) != BCJR_OK) return 0;
   const bool adjoint = (op == BCJR_OP_DENSE_BACKWARD || op == BCJR_OP_DENSE_BACKWARD_LAMBDA);
-  int grid = 0;
-  if (op == BCJR_OP_DENSE_BACKWARD_LAMBDA) {
-    int chunk = 0, parts = 0;
-    if (dlam_geometry(n_seq > 0 ? n_seq : 1, &grid, &chunk, &parts) != BCJR_OK) return 0;
-    return dense_layout(grid, seq_len, parts).total;
-  }
-  int clusters = 0;
-  if (dense_tc_clusters(adjoint, n_seq > 0 ? n_seq : 1, &clusters) != BCJR_OK) return 0;
-  return dense_tc_layout(adjoint, clusters, seq_len, n_seq > 0 ? n_seq : 1).total;
+  const bool dl = (op == BCJR_OP_DENSE_BACKWARD_LAMBDA);
+  const int N = n_seq > 0 ? n_seq : 1;
+  int clusters = 0, parts = 0;
+  if (dense_tc_clusters(adjoint, N, &clusters) != BCJR_OK) return 0;
+  if (dl && dlam_parts(&parts) != BCJR_OK) return 0;
+  const int chunk = dl ? clusters * bcjr::dense_tc_tile_seqs(adjoint) : N;
+  return dense_tc_layout(adjoint, clusters, seq_len, chunk < N ? chunk : N, dl ? parts : 0).total;
 }
 
 extern "C" {

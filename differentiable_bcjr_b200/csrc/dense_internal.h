@@ -9,34 +9,8 @@
 
 namespace bcjr {
 
-// Dense (fully connected) trellis: 256 states, 32 sequences per CTA.
+// Dense (fully connected) trellis: 256 states.
 constexpr int kDenseStates = 256;
-constexpr int kDenseRows = 32;
-
-struct DenseParams {
-  const float* w;          // [N][n]
-  const float* codebook;   // [S]
-  const float* g;          // [N][n] upstream gradient (backward)
-  const float* what_in;    // [N][n] soft codeword of the forward call (backward; centring)
-  float* w_hat;            // [N][n] (forward)
-  float* marginals;        // [N][n][S] or null (forward)
-  float* log_z;            // [N] or null (forward)
-  float* grad_w;           // [N][n] (backward)
-  float* gc_part;          // [grid][S] per-CTA codebook-gradient partials (backward)
-  const float* P;          // [S][S] exp(Lambda)
-  const float* PT;         // [S][S] its transpose
-  float* ckx;              // per CTA [n][32][S] normalised forward vectors
-  float* ckf;              // per CTA [n][32][S] forward adjoint accumulators (backward)
-  float* ckv;              // per CTA [n][32][S] rows V of the log-transition gradient, or null
-  float* ckw;              // per CTA [n][32][S] rows W of the log-transition gradient (with ckv)
-  float* mtab;             // per CTA [n][32] emission reference of each step
-  int* status;
-  size_t ck_stride;        // floats per CTA in ckx / ckf
-  size_t mt_stride;        // floats per CTA in mtab
-  float sc2;               // log2(e) / T
-  float two_over_T;
-  int n, N;
-};
 
 // The dense trellis on the tensor cores (dense_tc_kernel.cu): a cluster of
 // kDenseTCCluster CTAs per tile of kDenseTCRows MMA rows, CTA r holding K-slice
@@ -63,6 +37,15 @@ struct DenseTCParams {
   float* log_z;            // [N] or null (soft codeword)
   float* grad_w;           // [N][n] (vector-Jacobian product)
   float* gc_part;          // [clusters][S] codebook-gradient partials (vector-Jacobian product)
+  float* P;                // [S][S] exp(Lambda) row-major, or null (written by the prep kernel)
+  // Rows of the log-transition gradient (vector-Jacobian product, or null):
+  // per cluster a region of [n - 1][64 sequences][S] rows, row (t, q) for the
+  // transition t -> t + 1; each CTA writes its 64 states of every row.
+  float* rowX;
+  float* rowU;
+  float* rowV;
+  float* rowW;
+  size_t row_region;       // floats per cluster region of each row array
   int* status;
   size_t ck_stride;        // floats per CTA in ck and ckf
   size_t cks_stride;       // floats per CTA in cks
@@ -73,7 +56,7 @@ struct DenseTCParams {
 };
 
 // Log-transition gradient of the dense trellis (dense_dlam_kernel.cu): rows of
-// X, U, V, W written by the backward kernel, one region per backward CTA
+// X, U, V, W written by the tensor-core adjoint, one region per cluster
 // (`region_stride` floats apart), `spr` stages of 8 rows per region.
 struct DlamParams {
   const float* X;
@@ -87,13 +70,7 @@ struct DlamParams {
   long long total_stages;
 };
 
-// Launchers of the vector-Jacobian product that also writes the rows of the
-// log-transition gradient (dense_kernel.cu) and of that gradient's row sum
-// (dense_dlam_kernel.cu).
-size_t dense_smem_bytes();
-int dense_max_grid();
-cudaError_t launch_dense_prep(const float* lam, const DenseParams& p, cudaStream_t s);
-cudaError_t launch_dense(const DenseParams& p, const float* lam, int grid, cudaStream_t s, bool prep = true);
+// Launchers (dense_tc_kernel.cu, dense_dlam_kernel.cu).
 size_t dense_tc_smem_bytes();
 int dense_tc_max_clusters(bool adjoint);
 // Sequences per cluster tile: 128 for the soft codeword, 64 for the adjoint.

@@ -101,13 +101,15 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
 // the backward image holds P[n][k] (the product with P^T).  Each slice is
 // [K-chunk c][head, tail][256 rows n][8 k] in K-major core-matrix tiles.
 __global__ void dense_tc_prep_kernel(const float* __restrict__ lam, float* __restrict__ Bfwd,
-                                     float* __restrict__ Bbwd) {
+                                     float* __restrict__ Bbwd, float* __restrict__ Prow) {
   using namespace dtc;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= kS * kS) return;
   const int row = i / kS, col = i - row * kS;
+  const float pv = expf(lam[i]);  // P[row][col]
+  if (Prow) Prow[i] = pv;
   float hi, lo;
-  split_tf32(expf(lam[i]), hi, lo);  // P[row][col]
+  split_tf32(pv, hi, lo);
   auto put = [&](float* B, int nn, int kk) {
     const int r = kk / kSlice, c = (kk % kSlice) / 8, kc = (kk & 7) >> 2, e = kk & 3;
     unsigned char* base = reinterpret_cast<unsigned char*>(B) + static_cast<size_t>(r) * kBBytes + c * 2 * kBTile;
@@ -159,7 +161,9 @@ __global__ void dense_tc_mtab_kernel(const float* __restrict__ w, const float* _
   }
 }
 
-template <bool ADJ>
+// ADJ: the vector-Jacobian product instead of the soft codeword; ROWS (with
+// ADJ): also write the rows of the log-transition gradient.
+template <bool ADJ, bool ROWS>
 __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::kThreads, 1)
     dense_tc_kernel(const DenseTCParams p) {
   using namespace dtc;
@@ -690,8 +694,16 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
         const float inv = 1.f / sig;
         const float rden = static_cast<float>(1.0 / den);
         const float gsc = act ? gt : 0.f, tsc = act ? p.two_over_T : 0.f;
+        // Rows of the log-transition gradient: X_t = x_t / n, U_t = x_t (F~ + eps - D) / n
+        // for the transition t -> t + 1, with n = sum_p x_t(p) (P v_{t+1})(p) = sigma_{t+1} den_t;
+        // V, W of the transition t - 1 -> t are the next operand's two rows.
+        constexpr bool rows = ROWS;
+        const float rn = act ? static_cast<float>(1.0 / (static_cast<double>(sig) * den)) : 0.f;
+        const float ract = act ? 1.f : 0.f;
+        const size_t rbase = static_cast<size_t>(cid) * p.row_region + static_cast<size_t>(r * kSlice + c0);
         float gw = 0.f;
         float v1[16], v2[16];
+        float rx4[4], ru4[4];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const float xs = (j & 3) == 0 ? x4[j >> 2].x : (j & 3) == 1 ? x4[j >> 2].y : (j & 3) == 2 ? x4[j >> 2].z : x4[j >> 2].w;
@@ -707,6 +719,25 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
           const float d = wt - c;
           v1[j] = ex2f(-(d * d) * sc2 - mt) * z;
           v2[j] = v1[j] * (eps + bt);
+          if (rows && t < n - 1) {
+            rx4[j & 3] = xs * rn;
+            ru4[j & 3] = xs * (fs + eps - Dv) * rn;
+            if ((j & 3) == 3) {
+              const size_t o = rbase + (static_cast<size_t>(t) * kSeqs + qi) * kS + (j & ~3);
+              *reinterpret_cast<float4*>(p.rowX + o) = make_float4(rx4[0], rx4[1], rx4[2], rx4[3]);
+              *reinterpret_cast<float4*>(p.rowU + o) = make_float4(ru4[0], ru4[1], ru4[2], ru4[3]);
+            }
+          }
+        }
+        if (rows && t >= 1) {
+          const size_t o = rbase + (static_cast<size_t>(t - 1) * kSeqs + qi) * kS;
+#pragma unroll
+          for (int j = 0; j < 16; j += 4) {
+            *reinterpret_cast<float4*>(p.rowV + o + j) =
+                make_float4(ract * v1[j], ract * v1[j + 1], ract * v1[j + 2], ract * v1[j + 3]);
+            *reinterpret_cast<float4*>(p.rowW + o + j) =
+                make_float4(ract * v2[j], ract * v2[j + 1], ract * v2[j + 2], ract * v2[j + 3]);
+          }
         }
         *part_at(ptbase, t) = gw;
         if (t >= 1) put_pair(v1, v2);
@@ -775,15 +806,15 @@ namespace {
 // cluster occupancy queried once, so that later calls issue no driver queries
 // (a query can wait behind other users of the driver).  0 = not yet known.
 constexpr int kMaxDevices = 64;
-int g_tc_clusters[2][kMaxDevices] = {};
+int g_tc_clusters[3][kMaxDevices] = {};
 
-template <bool ADJ>
+template <bool ADJ, bool ROWS>
 int tc_clusters_of_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
-  if (dev < kMaxDevices && g_tc_clusters[ADJ][dev] > 0) return g_tc_clusters[ADJ][dev];
+  if (dev < kMaxDevices && g_tc_clusters[ADJ + ROWS][dev] > 0) return g_tc_clusters[ADJ + ROWS][dev];
   const size_t smem = dense_tc_smem_bytes();
-  if (cudaFuncSetAttribute(dense_tc_kernel<ADJ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(dense_tc_kernel<ADJ, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return 0;
   int sms = 0;
@@ -793,19 +824,20 @@ int tc_clusters_of_device() {
   cfg.blockDim = dim3(dtc::kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   int clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&clusters, dense_tc_kernel<ADJ>, &cfg) != cudaSuccess) return 0;
-  if (dev < kMaxDevices) g_tc_clusters[ADJ][dev] = clusters;
+  if (cudaOccupancyMaxActiveClusters(&clusters, dense_tc_kernel<ADJ, ROWS>, &cfg) != cudaSuccess) return 0;
+  if (dev < kMaxDevices) g_tc_clusters[ADJ + ROWS][dev] = clusters;
   return clusters;
 }
 }  // namespace
 
 int dense_tc_max_clusters(bool adjoint) {
-  return adjoint ? tc_clusters_of_device<true>() : tc_clusters_of_device<false>();
+  // the row-writing variant has the same resources as the plain adjoint
+  return adjoint ? tc_clusters_of_device<true, false>() : tc_clusters_of_device<false, false>();
 }
 
 cudaError_t launch_dense_tc(const DenseTCParams& p, const float* lam, bool adjoint, int clusters, cudaStream_t s) {
   using namespace dtc;
-  dense_tc_prep_kernel<<<(kS * kS + 255) / 256, 256, 0, s>>>(lam, p.Bfwd, p.Bbwd);
+  dense_tc_prep_kernel<<<(kS * kS + 255) / 256, 256, 0, s>>>(lam, p.Bfwd, p.Bbwd, p.P);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const long long total = static_cast<long long>(p.N) * p.n;
@@ -813,11 +845,17 @@ cudaError_t launch_dense_tc(const DenseTCParams& p, const float* lam, bool adjoi
   dense_tc_mtab_kernel<<<static_cast<unsigned>(blocks < 4096 ? blocks : 4096), kS, 0, s>>>(p.w, p.codebook, p.sc2, total,
                                                                                          p.mtab);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (dense_tc_max_clusters(adjoint) < 1) return cudaErrorNotSupported;  // also sets the shared-memory attribute
-  if (adjoint) {
-    dense_tc_kernel<true><<<clusters * kCL, kThreads, dense_tc_smem_bytes(), s>>>(p);
+  // the occupancy queries also set the kernels' shared-memory attribute
+  const bool rows = adjoint && p.rowX != nullptr;
+  if (rows) {
+    if (tc_clusters_of_device<true, true>() < 1) return cudaErrorNotSupported;
+    dense_tc_kernel<true, true><<<clusters * kCL, kThreads, dense_tc_smem_bytes(), s>>>(p);
+  } else if (adjoint) {
+    if (tc_clusters_of_device<true, false>() < 1) return cudaErrorNotSupported;
+    dense_tc_kernel<true, false><<<clusters * kCL, kThreads, dense_tc_smem_bytes(), s>>>(p);
   } else {
-    dense_tc_kernel<false><<<clusters * kCL, kThreads, dense_tc_smem_bytes(), s>>>(p);
+    if (tc_clusters_of_device<false, false>() < 1) return cudaErrorNotSupported;
+    dense_tc_kernel<false, false><<<clusters * kCL, kThreads, dense_tc_smem_bytes(), s>>>(p);
   }
   return cudaGetLastError();
 }

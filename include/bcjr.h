@@ -188,7 +188,10 @@ bcjr_status viterbi_decode(const float* w, const float* codebook, int state_bits
  * row = source state.  Same outputs and conventions as the bitshift calls.
  * Supported: n_states = 256.  Every step's forward vector is kept (no recompute
  * schedule), so checkpoint_interval must be 0 or 1; the workspace holds 32 KiB
- * per step per 32 sequences in flight (two such areas for the backward call).
+ * per step per 128 sequences in flight for the forward call and 32 KiB per step
+ * per 64 sequences in flight for the backward call (sequences in flight: up to
+ * 128 x 33 and 64 x 33 on a B200).  The per-step contractions run on the
+ * tensor cores in three-pass tf32 (float32-level accuracy).
  */
 bcjr_status bcjr_dense_forward(const float* w, const float* codebook, const float* log_trans,
                                float T, int n_states, int seq_len, int n_seq, float* w_hat,
@@ -211,9 +214,9 @@ bcjr_status bcjr_dense_backward(const float* grad_w_hat, const float* w, const f
  * grad_log_trans are added to, otherwise overwritten.  The sum over
  * (sequence, transition) rows runs on the tensor cores in three-pass tf32
  * (float32-level accuracy).  Workspace: bcjr_workspace_size(BCJR_OP_DENSE_BACKWARD_LAMBDA, ...),
- * which adds two more 32 KiB rows per step per 32 sequences in flight and a
- * 256 KiB partial sum per SM; batches longer than 32 sequences per resident
- * CTA run in several launches inside the call.
+ * which adds four 64 KiB rows per step per 64 sequences in flight and a 256 KiB
+ * partial sum per SM; batches longer than one 64-sequence tile per resident
+ * cluster run in several launches inside the call.
  */
 bcjr_status bcjr_dense_backward_lambda(const float* grad_w_hat, const float* w, const float* codebook,
                                        const float* log_trans, const float* w_hat, float T, int n_states,

@@ -4,7 +4,7 @@ bcjr_dense_backward_lambda returns dL/dLambda next to the usual VJP; the sum
 over (sequence, transition) rows runs on the tcgen05 tensor cores in
 three-pass tf32.  Checked against the float64 oracle (itself pinned to path
 enumeration and finite differences) at lengths 1 (no transitions: zero), 2, 7
-and 64, batches that fill one CTA, leave a ragged tail and span several CTAs;
+and 64, batches that fill one tile, leave a ragged tail and span several tiles;
 against the zero-sum invariant (a common shift of Lambda changes no path's
 probability); and, for a batch longer than one launch, against the sum of the
 two halves computed separately.
@@ -43,11 +43,10 @@ def test_log_transition_gradient_parity(B, n, N, T):
     gw, gc, gl = B.bcjr_dense_backward(dg, dw, dc, dl, w_hat, T, want_grad_log_trans=True)
     gw0, gc0 = B.bcjr_dense_backward(dg, dw, dc, dl, w_hat, T)
     torch.cuda.synchronize()
-    # The extra output leaves the others unchanged up to float32 rounding: the
-    # plain call runs the tensor-core adjoint, this one the kernel that also
-    # writes the rows of the log-transition gradient.
-    assert_rel_l2(gw, to_np(gw0), 1e-5, "grad_w of the two calls")
-    assert_rel_l2(gc, to_np(gc0), 1e-5, "grad_codebook of the two calls")
+    # the extra output changes nothing in the others (one launch: the same
+    # kernel, tiles and reduction order as the plain call)
+    assert torch.equal(gw, gw0)
+    assert torch.equal(gc, gc0)
     o_gw, o_gc, o_gl = oracle.dense_backward(g, w, c, lam, T, want_grad_lam=True)
     assert_rel_l2(gw0, o_gw, GRAD_REL_L2, "grad_w (plain call)")
     assert_rel_l2(gc0, o_gc, GRAD_REL_L2, "grad_codebook (plain call)")
@@ -78,8 +77,9 @@ def test_log_transition_gradient_sums_to_zero_and_repeats(B):
 
 
 def test_log_transition_gradient_over_several_launches(B):
-    # More sequences than one launch holds (32 per resident CTA): the call runs
-    # in chunks and accumulates; compare with the two halves computed apart.
+    # More sequences than one launch holds (one 64-sequence tile per resident
+    # cluster): the call runs in chunks and accumulates; compare with the two
+    # halves computed apart.
     B.lib()
     n, T = 3, 0.4
     import ctypes
@@ -127,16 +127,17 @@ def test_dense_autograd_function(B):
     lv2 = lam.cuda()
     w2 = w.cuda().requires_grad_(True)
     (B.dense_soft_quantize(w2, c.cuda(), lv2, T) * g.cuda()).sum().backward()
-    assert_rel_l2(w2.grad, o_gw, GRAD_REL_L2, "grad_w (plain call)")
-    assert_rel_l2(w2.grad, to_np(wv.grad), 1e-5, "grad_w of the two calls")
+    assert torch.equal(w2.grad, wv.grad)
 
 
 @pytest.mark.slow
 def test_log_transition_gradient_full_workload(B):
     # 4096 sequences x 4096 steps (the dense workload): the oracle cannot run
     # at this size, so check what holds at any size -- the zero sum, agreement
-    # of the other outputs with the plain backward call (a different kernel:
-    # float32-level agreement), run-to-run identity.
+    # of the other outputs with the plain backward call (grad_w bit for bit;
+    # grad_codebook to float32 rounding, since this call runs the tiles in two
+    # launches and adds their codebook partials in another order), run-to-run
+    # identity.
     W = I.WORKLOADS["dense_S256"]
     n, N, T = W["seq_len"], W["n_seq"], W["T"][0]
     c, w, g, lam = I.codebook(S).cuda(), I.weights(N, n).cuda(), I.upstream_grad(N, n).cuda(), I.log_transition(S).cuda()
@@ -145,7 +146,7 @@ def test_log_transition_gradient_full_workload(B):
     gw0, gc0 = B.bcjr_dense_backward(g, w, c, lam, w_hat, T)
     _, _, gl2 = B.bcjr_dense_backward(g, w, c, lam, w_hat, T, want_grad_log_trans=True)
     torch.cuda.synchronize()
-    assert_rel_l2(gw, to_np(gw0), 1e-5, "grad_w of the two calls")
+    assert torch.equal(gw, gw0)
     assert_rel_l2(gc, to_np(gc0), 1e-5, "grad_codebook of the two calls")
     assert torch.equal(gl, gl2)
     x = gl.double()
