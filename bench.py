@@ -63,7 +63,7 @@ def parse():
     ap.add_argument("--n-seq", type=int, default=0,
                     help="sequences per GPU (default: the workload's 65536); smaller only for profiling")
     ap.add_argument("--workload", default="projection",
-                    choices=["projection", "dense", "viterbi", "bitwidth", "mufu"],
+                    choices=["projection", "dense", "viterbi", "bitwidth", "mufu", "tcprobe"],
                     help="projection: the S=2^16, k=2 headline; dense: the 256-state fully connected trellis; "
                          "viterbi: hard decode of the projection; bitwidth: k = 2, 3, 4 at S=2^16 on "
                          "16384 sequences (forward, backward and hard decode per k); mufu: throughput of the "
@@ -447,6 +447,41 @@ def run_mufu(args):
             "ex2_ops_per_clk_per_sm": per["ex2"], "lg2_ops_per_clk_per_sm": per["lg2"],
             "spread_over_sms": {op: [rs[0]["min"], rs[0]["max"]] for op, rs in res.items()},
             "gpu_launches": 2 * max(args.steps, 1) + max(args.warmup, 1)}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_tcprobe(args):
+    """The two costs that bound a step of the dense tensor-core kernels: the
+    issue cost of a tf32 tensor-core product by N, and the st.async exchange
+    bandwidth between the CTAs of 4-CTA clusters (all SMs, and a few)."""
+    world, rank, local = dist_env()
+    if rank != 0:
+        return 0
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import differentiable_bcjr_b200 as B
+    iters, reps, rounds = 4096, 4, 100
+    for _ in range(max(args.warmup, 1)):
+        B.probe_mma_tf32(64, iters, dev)
+        B.probe_dsmem(reps, rounds, 0, dev)
+    steps = max(args.steps, 1)
+    mma = {n: statistics.median(B.probe_mma_tf32(n, iters, dev)["clk_per_mma"] for _ in range(steps))
+           for n in (16, 32, 64, 128, 256)}
+    xall = [B.probe_dsmem(reps, rounds, 0, dev) for _ in range(steps)]
+    xfew = [B.probe_dsmem(reps, rounds, 2, dev) for _ in range(steps)]
+    bw_all = statistics.median(x["bytes_per_clk_per_sm"] for x in xall)
+    bw_few = statistics.median(x["bytes_per_clk_per_sm"] for x in xfew)
+    line = {"metric": "tcgen05 tf32 product issue cost (M=128, K=8, A in tensor memory) and 4-CTA-cluster "
+                      "st.async exchange bandwidth",
+            "value": bw_all, "unit": "bytes/clk/SM", "n_gpus": 1, "steps": steps, "warmup": args.warmup,
+            "higher_is_better": True, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "tc_probe", "mma_iters": iters, "dsmem_reps": reps, "dsmem_rounds": rounds,
+                       "dsmem_ctas_all": xall[0]["ctas"], "dsmem_ctas_few": xfew[0]["ctas"]},
+            "mma_clk_per_product": {str(n): c for n, c in mma.items()},
+            "mma_mac_per_clk_per_sm": {str(n): 128.0 * n * 8 / c for n, c in mma.items()},
+            "dsmem_bytes_per_clk_per_sm": {"all_sms": bw_all, "two_clusters": bw_few},
+            "gpu_launches": 5 * steps + 2 * steps + 2 * max(args.warmup, 1)}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -844,6 +879,8 @@ def main():
         return run_viterbi(args)
     if args.workload == "bitwidth":
         return run_bitwidth(args)
+    if args.workload == "tcprobe":
+        return run_tcprobe(args)
     if args.workload == "mufu":
         return run_mufu(args)
     return run_gpu(args)

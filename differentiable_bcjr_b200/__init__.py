@@ -24,7 +24,7 @@ __all__ = [
     "LIB_PATH", "lib", "BCJRError", "bcjr_forward", "bcjr_backward", "viterbi_decode",
     "bcjr_dense_forward", "bcjr_dense_backward", "workspace_size", "Workspace",
     "SoftTrellisQuant", "soft_quantize", "DenseTrellisQuant", "dense_soft_quantize", "bcjr_forward_static_scratch",
-    "static_scratch_status", "probe_xu", "OP_FORWARD", "OP_BACKWARD", "OP_VITERBI",
+    "static_scratch_status", "probe_xu", "probe_mma_tf32", "probe_dsmem", "OP_FORWARD", "OP_BACKWARD", "OP_VITERBI",
     "OP_DENSE_FORWARD", "OP_DENSE_BACKWARD", "OP_DENSE_BACKWARD_LAMBDA", "STATUS",
 ]
 
@@ -68,6 +68,8 @@ _SIGS = {
     "bcjr_static_scratch_status": (_I, [_P]),
     "bcjr_status_string": (ctypes.c_char_p, [_I]),
     "bcjr_probe_xu": (_I, [_I, _I, _P, _P, _I, _P]),
+    "bcjr_probe_mma_tf32": (_I, [_I, _I, _P, _P, _I, _P]),
+    "bcjr_probe_dsmem": (_I, [_I, _I, _P, _P, _I, _P]),
     "bcjr_version": (_I, []),
 }
 
@@ -391,3 +393,44 @@ def probe_xu(op: str = "ex2", iters: int = 4096, device=None) -> dict:
     rates = sorted(ops / float(c) for c in cycles.cpu().tolist())
     return {"ops_per_clk_per_sm": rates[len(rates) // 2], "min": rates[0], "max": rates[-1], "sms": sms,
             "ops": ops * sms}
+
+
+def probe_mma_tf32(n: int = 64, iters: int = 4096, device=None) -> dict:
+    """Issue cost of one tcgen05 tf32 product with operand A in tensor memory
+    (bcjr_probe.h), M = 128, K = 8 and the given N, one CTA per SM.  Returns
+    {"clk_per_mma", "mac_per_clk_per_sm"} (medians over SMs), "sms"."""
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    cycles = torch.zeros(sms, dtype=torch.int64, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().bcjr_probe_mma_tf32(int(n), int(iters), _ptr(cycles), _ptr(status), sms, _stream(dev)),
+               "bcjr_probe_mma_tf32")
+        torch.cuda.synchronize(dev)
+    if int(status.item()) != 0:
+        raise BCJRError(int(status.item()), "bcjr_probe_mma_tf32: a wait ran out")
+    c = sorted(float(v) for v in cycles.cpu().tolist())
+    med = c[len(c) // 2]
+    return {"clk_per_mma": med / iters, "mac_per_clk_per_sm": 128.0 * n * 8 * iters / med, "sms": sms}
+
+
+def probe_dsmem(reps: int = 4, rounds: int = 100, clusters: int = 0, device=None) -> dict:
+    """Bandwidth of the st.async exchange between the CTAs of 4-CTA clusters
+    (bcjr_probe.h).  clusters = 0: one per 4 SMs.  Returns
+    {"bytes_per_clk_per_sm": median over CTAs of the bytes each sends per clock,
+    "min", "max", "ctas"}."""
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    ncl = int(clusters) if clusters > 0 else sms // 4
+    cycles = torch.zeros(4 * ncl, dtype=torch.int64, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib().bcjr_probe_dsmem(int(reps), int(rounds), _ptr(cycles), _ptr(status), ncl, _stream(dev)),
+               "bcjr_probe_dsmem")
+        torch.cuda.synchronize(dev)
+    if int(status.item()) != 0:
+        raise BCJRError(int(status.item()), "bcjr_probe_dsmem: a wait ran out")
+    out = 3 * 32768 * int(reps) * int(rounds)
+    r = sorted(out / float(v) for v in cycles.cpu().tolist())
+    return {"bytes_per_clk_per_sm": r[len(r) // 2], "min": r[0], "max": r[-1], "ctas": 4 * ncl}
+
