@@ -111,6 +111,25 @@ def _need_cuda(*ts):
             raise ValueError("tensors must be contiguous")
 
 
+def _expect(t, name, shape, dtype, device):
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, not {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, not {t.dtype}")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the weights on {device}")
+
+
+def _weights_2d(w):
+    if w.dim() != 2:
+        raise ValueError("w must be [n_seq][seq_len]")
+    if w.dtype != torch.float32:
+        raise ValueError(f"w must be torch.float32, not {w.dtype}")
+    return w.shape
+
+
 def _ptr(t):
     return None if t is None else t.data_ptr()
 
@@ -158,10 +177,12 @@ def bcjr_forward(w, codebook, T, state_bits, k, want_marginals=False, checkpoint
     """Soft codeword of every row of w [N][n] (float32, CUDA).  Returns
     (w_hat [N][n], marginals [N][n][S] or None, log_z [N]).
     `timeout_probe_cycles` is the testing aid of bcjr_options (see bcjr.h)."""
-    _need_cuda(w, codebook)
-    N, n = w.shape
+    _need_cuda(w, codebook, out)
+    N, n = _weights_2d(w)
     S = 1 << state_bits
     dev = w.device
+    _expect(codebook, "codebook", (S,), torch.float32, dev)
+    _expect(out, "out", (N, n), torch.float32, dev)
     w_hat = out if out is not None else torch.empty((N, n), dtype=torch.float32, device=dev)
     marg = torch.empty((N, n, S), dtype=torch.float32, device=dev) if want_marginals else None
     log_z = torch.empty((N,), dtype=torch.float32, device=dev)
@@ -177,17 +198,6 @@ def bcjr_forward(w, codebook, T, state_bits, k, want_marginals=False, checkpoint
 
 
 STATIC_SCRATCH_BYTES = 32 << 20
-
-
-def _expect(t, name, shape, dtype, device):
-    if t is None:
-        return
-    if tuple(t.shape) != tuple(shape):
-        raise ValueError(f"{name} must have shape {tuple(shape)}, not {tuple(t.shape)}")
-    if t.dtype != dtype:
-        raise ValueError(f"{name} must be {dtype}, not {t.dtype}")
-    if t.device != device:
-        raise ValueError(f"{name} is on {t.device}, the weights on {device}")
 
 
 def bcjr_forward_static_scratch(w, codebook, T, state_bits, k, w_hat, log_z=None, marginals=None,
@@ -228,9 +238,13 @@ def bcjr_backward(grad_w_hat, w, codebook, w_hat, T, state_bits, k, checkpoint_i
                   grad_codebook=None, accumulate_codebook=False, sequences_in_flight=0, grad_w_out=None):
     """VJP of the soft codeword.  Returns (grad_w [N][n], grad_codebook [S]); grad_w goes
     into `grad_w_out` when given."""
-    _need_cuda(grad_w_hat, w, codebook, w_hat, grad_w_out)
-    N, n = w.shape
+    _need_cuda(grad_w_hat, w, codebook, w_hat, grad_w_out, grad_codebook)
+    N, n = _weights_2d(w)
     S = 1 << state_bits
+    for t, name, shape in ((grad_w_hat, "grad_w_hat", (N, n)), (w_hat, "w_hat", (N, n)),
+                           (grad_w_out, "grad_w_out", (N, n)), (codebook, "codebook", (S,)),
+                           (grad_codebook, "grad_codebook", (S,))):
+        _expect(t, name, shape, torch.float32, w.device)
     dev = w.device
     grad_w = grad_w_out if grad_w_out is not None else torch.empty((N, n), dtype=torch.float32, device=dev)
     if grad_codebook is None:
@@ -250,7 +264,8 @@ def bcjr_backward(grad_w_hat, w, codebook, w_hat, T, state_bits, k, checkpoint_i
 def viterbi_decode(w, codebook, state_bits, k, ws=None):
     """Hard (T -> 0) decode.  Returns (states int32 [N][n], w_hard [N][n])."""
     _need_cuda(w, codebook)
-    N, n = w.shape
+    N, n = _weights_2d(w)
+    _expect(codebook, "codebook", (1 << state_bits,), torch.float32, w.device)
     dev = w.device
     states = torch.empty((N, n), dtype=torch.int32, device=dev)
     w_hard = torch.empty((N, n), dtype=torch.float32, device=dev)
@@ -272,8 +287,10 @@ def _log2_states(S: int) -> int:
 
 def bcjr_dense_forward(w, codebook, log_trans, T, want_marginals=False, checkpoint_interval=0, ws=None):
     _need_cuda(w, codebook, log_trans)
-    N, n = w.shape
+    N, n = _weights_2d(w)
     S = codebook.shape[0]
+    _expect(codebook, "codebook", (S,), torch.float32, w.device)
+    _expect(log_trans, "log_trans", (S, S), torch.float32, w.device)
     dev = w.device
     w_hat = torch.empty((N, n), dtype=torch.float32, device=dev)
     marg = torch.empty((N, n, S), dtype=torch.float32, device=dev) if want_marginals else None
@@ -296,8 +313,12 @@ def bcjr_dense_backward(grad_w_hat, w, codebook, log_trans, w_hat, T, checkpoint
     `grad_codebook` / `grad_log_trans` tensors, the results go there, added to
     their contents when `accumulate` is set."""
     _need_cuda(grad_w_hat, w, codebook, log_trans, w_hat, grad_codebook, grad_log_trans)
-    N, n = w.shape
+    N, n = _weights_2d(w)
     S = codebook.shape[0]
+    for t, name, shape in ((grad_w_hat, "grad_w_hat", (N, n)), (w_hat, "w_hat", (N, n)), (codebook, "codebook", (S,)),
+                           (log_trans, "log_trans", (S, S)), (grad_codebook, "grad_codebook", (S,)),
+                           (grad_log_trans, "grad_log_trans", (S, S))):
+        _expect(t, name, shape, torch.float32, w.device)
     dev = w.device
     grad_w = torch.empty((N, n), dtype=torch.float32, device=dev)
     if grad_codebook is None or (want_grad_log_trans and grad_log_trans is None):
