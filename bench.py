@@ -680,9 +680,10 @@ def run_dense(args):
         if e2e is not None:
             line["e2e"] = e2e
         if world == 1 and not args.no_cpu_baseline:
-            rate, threads, dt = dense_oracle_rate(max(1, min(len(os.sched_getaffinity(0)), 16)), 256, T)
+            # whole sequences of the workload (4096 steps): about 15 s of CPU work on 16 cores
+            rate, threads, dt = dense_oracle_rate(max(1, min(len(os.sched_getaffinity(0)), 16)), n, T)
             line["cpu_baseline"] = {"value": rate, "unit": "weights/s", "cores": threads, "kind": "oracle",
-                                    "sample": f"{threads} sequences x 256 steps of the workload (fwd+bwd), "
+                                    "sample": f"{threads} whole sequences ({n} steps) of the workload (fwd+bwd), "
                                               f"{dt:.1f} s of CPU work"}
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -795,12 +796,18 @@ def run_viterbi(args):
         if world == 1 and not args.no_cpu_baseline:
             import oracle
             cores = len(os.sched_getaffinity(0))
-            sample = max(1, min(cores, 16))
-            wq = I.weights(sample, n)
-            t0 = time.perf_counter()
-            oracle.viterbi(wq, c_h, L, k, nthreads=min(cores, sample))
-            dt = time.perf_counter() - t0
-            line["cpu_baseline"] = {"value": sample * n / dt, "unit": "weights/s", "cores": min(cores, sample),
+            threads = max(1, min(cores, 16))
+            # grow the sample (whole sequences of the workload) to about 10 s of CPU work
+            sample, dt = threads, 0.0
+            while True:
+                wq = I.weights(sample, n)
+                t0 = time.perf_counter()
+                oracle.viterbi(wq, c_h, L, k, nthreads=threads)
+                dt = time.perf_counter() - t0
+                if dt >= 10.0 or sample >= 65536:
+                    break
+                sample = min(65536, sample * max(2, int(10.0 / max(dt, 1e-3))))
+            line["cpu_baseline"] = {"value": sample * n / dt, "unit": "weights/s", "cores": threads,
                                     "kind": "oracle", "sample": f"{sample} whole sequences, {dt:.1f} s of CPU work"}
         print(json.dumps(line), flush=True)
     if world > 1:
