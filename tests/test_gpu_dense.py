@@ -1,11 +1,12 @@
 """GPU parity of the dense-trellis calls with the float64 oracle (needs a B200).
 
 Shapes: 256 states (the size the kernels are built for); sequence counts
-that fill one CTA of the backward kernel, leave a ragged tail (40 = 32 + 8)
-and span several CTAs, and for the forward call's 128-sequence cluster tiles
-a tile plus one (129), a ragged third tile (300) and more tiles than
-resident clusters (2100); lengths 1 (a plain softmax per sequence), 2, 7,
-16, 33 and 64; several temperatures.  The
+against the cluster tiles (128 sequences in the soft-codeword call, 64 in the
+vector-Jacobian product): part of one tile (3, 40), a tile plus a ragged
+rest (70, 129), several tiles (300, 2100), and more tiles than the 33
+clusters that fit at once in both calls (4300: 34 and 68 tiles, so clusters
+run several tiles in turn); lengths 1 (a plain softmax per sequence), 2, 3,
+7, 16, 33 and 64; several temperatures.  The
 full dense workload (4096 sequences of 4096 steps) is checked on sampled
 sequences and by the translation identity.
 """
@@ -36,7 +37,7 @@ def _case(n, N, seed):
 
 
 @pytest.mark.parametrize("n,N,T", [(1, 3, 0.5), (7, 40, 0.2), (64, 40, 1.0), (64, 70, 0.2), (2, 129, 0.3),
-                                   (33, 300, 0.2), (16, 2100, 0.5)])
+                                   (33, 300, 0.2), (16, 2100, 0.5), (3, 4300, 0.3)])
 def test_dense_parity(B, n, N, T):
     c, w, g, lam = _case(n, N, seed=n + N)
     dc, dw, dg, dl = c.cuda(), w.cuda(), g.cuda(), lam.cuda()
