@@ -1,5 +1,7 @@
-// dense_tc_kernel.cu -- soft codeword of the dense (fully connected) trellis on
-// the fifth-generation tensor cores (tcgen05, sm_100a).
+// dense_tc_kernel.cu -- the dense (fully connected) trellis on the
+// fifth-generation tensor cores (tcgen05, sm_100a): the soft codeword with its
+// marginals and log Z, the vector-Jacobian product, and the rows of the
+// log-transition gradient.
 //
 // "BCJR-QAT: A Differentiable Relaxation of Trellis-Coded Weight Quantization",
 // abstract: the relaxation is a 1D Ising-like chain solved by a transfer
@@ -13,30 +15,37 @@
 // cancels in gamma, and dividing by the previous step's sum keeps every row's
 // sum in (0, 1] (P is row-stochastic for the normalised Lambda, and within a
 // step's column-sum spread in general).  log2 Z = sum_t m_t + sum_t log2 s_t.
+// The vector-Jacobian product ("key technical innovations": exact gradients)
+// runs the same recursions on a second operand per sequence, u (.) (F~ + eps)
+// and v (.) (eps + B~), whose ratios to the first give the centred
+// accumulators F~ and B~.
 //
-// Each step is one [rows x 256] x [256 x 256] contraction: a real batched
+// Each step is one [128 x 256] x [256 x 256] contraction: a real batched
 // matrix product, run here as three tf32 products (x = hi + lo, hi*hi + hi*lo +
 // lo*hi: float32-level accuracy; one tf32 product would leave ~5e-4 relative
 // error in a step's dominant terms).
 //
-// Work split.  A thread-block cluster of 4 CTAs owns 128 sequences (the MMA's
-// M = 128).  CTA r keeps K-slice r of the transfer matrix (input states
-// 64r .. 64r+63, as tf32 head and tail in K-major core-matrix tiles, 128 KiB)
-// resident in shared memory; its operand A, the same 64 states of the current
-// vector as head and tail, lives in tensor memory next to the accumulator.
-// The 96 MMAs of a step (4 output blocks of 64 states x 8 K-chunks x 3
-// products) give partial sums for all 256 output states; CTA r's output states
-// 64r .. 64r+63 are exactly its next K-slice, so only the partial sums cross
-// CTAs (a reduce-scatter over distributed shared memory) and the operand never
-// does.  The output blocks are issued and committed one at a time, the other
-// CTAs' blocks first, so sending a finished block (st.async from the sending
-// warps' registers, completing on the receiver's mbarrier) overlaps the MMAs
-// of the next.  Four warps own the CTA's 64 output states of one row each:
-// they add the three received blocks to their own, scale and store the new
-// vector, and write it back to tensor memory as the next operand.  Each row's
-// sum over the CTA's states rides along with the next step's blocks (for the
-// next normalisation).  A split cluster barrier per step keeps a CTA from
-// overwriting a receive buffer that another CTA is still reading.  The
+// Work split.  A thread-block cluster of 4 CTAs owns a tile of 128 MMA rows:
+// 128 sequences (soft codeword) or 64 sequences with their two operands on
+// adjacent rows (vector-Jacobian product).  CTA r keeps K-slice r of the
+// transfer matrix (input states 64r .. 64r+63, as tf32 head and tail in
+// K-major core-matrix tiles, 128 KiB) resident in shared memory; its operand
+// A, the same 64 states of the current vectors as head and tail, lives in
+// tensor memory next to the accumulator.  The 96 MMAs of a step (4 output
+// blocks of 64 states x 8 K-chunks x 3 products) give partial sums for all 256
+// output states; CTA r's output states 64r .. 64r+63 are exactly its next
+// K-slice, so only the partial sums cross CTAs (a reduce-scatter over
+// distributed shared memory) and the operand never does.  A ninth warp issues
+// the MMAs and commits the output blocks one at a time, the other CTAs'
+// blocks first; each of the eight worker warps (two per tensor-memory lane
+// quadrant, 32 states of a row each) sends its half of a finished block with
+// st.async from registers, completing on the receiver's mbarrier, while the
+// MMAs of the next block run.  The workers then add the three received halves
+// to their own, scale, store and write the new operand back to tensor memory.
+// The row sums for the next normalisation come from the tensor cores too (the
+// operand times a tile of ones, issued after the first block) and travel to
+// the other CTAs on their own.  A split cluster barrier per step keeps a CTA
+// from overwriting a receive buffer that another CTA is still reading.  The
 // backward sweep reloads the resident slice with P's other orientation.  The
 // per-step reference m_t comes from a small kernel that finds each weight's
 // nearest codeword.
@@ -226,7 +235,7 @@ __global__ void __cluster_dims__(kDenseTCCluster, 1, 1) __launch_bounds__(dtc::k
     ph ^= 1u;
   };
 
-  // Load a resident slice (tid 0), completing on bar_b.
+  // Load a resident slice (thread 0), completing on bar_b.
   auto load_b = [&](const float* image) {
     if (tid == 0) {
       mbar_arm(bar_b, kBBytes);
