@@ -70,6 +70,7 @@ _SIGS = {
     "bcjr_probe_xu": (_I, [_I, _I, _P, _P, _I, _P]),
     "bcjr_probe_mma_tf32": (_I, [_I, _I, _P, _P, _I, _P]),
     "bcjr_probe_dsmem": (_I, [_I, _I, _P, _P, _I, _P]),
+    "bcjr_probe_dsmem_bulk": (_I, [_I, _I, _I, _P, _P, _I, _P]),
     "bcjr_version": (_I, []),
 }
 
@@ -435,22 +436,28 @@ def probe_mma_tf32(n: int = 64, iters: int = 4096, device=None) -> dict:
     return {"clk_per_mma": med / iters, "mac_per_clk_per_sm": 128.0 * n * 8 * iters / med, "sms": sms}
 
 
-def probe_dsmem(reps: int = 4, rounds: int = 100, clusters: int = 0, device=None) -> dict:
-    """Bandwidth of the st.async exchange between the CTAs of 4-CTA clusters
-    (bcjr_probe.h).  clusters = 0: one per 4 SMs.  Returns
-    {"bytes_per_clk_per_sm": median over CTAs of the bytes each sends per clock,
-    "min", "max", "ctas"}."""
+def probe_dsmem(reps: int = 4, rounds: int = 100, clusters: int = 0, device=None, chunk: int = 0) -> dict:
+    """Bandwidth of the exchange between the CTAs of 4-CTA clusters
+    (bcjr_probe.h): per-thread st.async stores (chunk = 0) or bulk copies of
+    `chunk` bytes (bcjr_probe_dsmem_bulk).  clusters = 0: one per 4 SMs.
+    Returns {"bytes_per_clk_per_sm": median over CTAs of the bytes each sends
+    per clock, "min", "max", "ctas"}."""
     dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     ncl = int(clusters) if clusters > 0 else sms // 4
     cycles = torch.zeros(4 * ncl, dtype=torch.int64, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
+    name = "bcjr_probe_dsmem_bulk" if chunk else "bcjr_probe_dsmem"
     with torch.cuda.device(dev):
-        _check(lib().bcjr_probe_dsmem(int(reps), int(rounds), _ptr(cycles), _ptr(status), ncl, _stream(dev)),
-               "bcjr_probe_dsmem")
+        if chunk:
+            rc = lib().bcjr_probe_dsmem_bulk(int(chunk), int(reps), int(rounds), _ptr(cycles), _ptr(status), ncl,
+                                             _stream(dev))
+        else:
+            rc = lib().bcjr_probe_dsmem(int(reps), int(rounds), _ptr(cycles), _ptr(status), ncl, _stream(dev))
+        _check(rc, name)
         torch.cuda.synchronize(dev)
     if int(status.item()) != 0:
-        raise BCJRError(int(status.item()), "bcjr_probe_dsmem: a wait ran out")
+        raise BCJRError(int(status.item()), name + ": a wait ran out")
     out = 3 * 32768 * int(reps) * int(rounds)
     r = sorted(out / float(v) for v in cycles.cpu().tolist())
     return {"bytes_per_clk_per_sm": r[len(r) // 2], "min": r[0], "max": r[-1], "ctas": 4 * ncl}

@@ -250,7 +250,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
     }
   }
 }
-// st.async of one float64 / two float64 / one float32 into cluster shared
+// st.async of one or two float64, or of one, two or four float32, into cluster shared
 // memory at `raddr`, completing their bytes on the mbarrier at `rbar` (both
 // addresses already mapped to the destination CTA).
 __device__ __forceinline__ void st_async_f64(uint32_t raddr, double v, uint32_t rbar) {
@@ -271,6 +271,12 @@ __device__ __forceinline__ void st_async_f32(uint32_t raddr, float v, uint32_t r
 __device__ __forceinline__ void st_async_v2f32(uint32_t raddr, float a, float b, uint32_t rbar) {
   asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(raddr),
                "f"(a), "f"(b), "r"(rbar)
+               : "memory");
+}
+__device__ __forceinline__ void st_async_v4f32(uint32_t raddr, float a, float b, float c, float d, uint32_t rbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   raddr),
+               "f"(a), "f"(b), "f"(c), "f"(d), "r"(rbar)
                : "memory");
 }
 // Split cluster barrier without memory ordering: it only orders the

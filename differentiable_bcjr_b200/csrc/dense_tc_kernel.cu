@@ -90,12 +90,6 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTAh = kS, kTAl = kS + kSlice, kTSum = kS + 2 * kSlice;
 constexpr uint32_t kIdescN64 = idesc_tf32(64), kIdescN16 = idesc_tf32(16);
 
-__device__ __forceinline__ void st_async_v4f32(uint32_t raddr, float a, float b, float c, float d, uint32_t rbar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-                   raddr),
-               "f"(a), "f"(b), "f"(c), "f"(d), "r"(rbar)
-               : "memory");
-}
 // Bulk copy global -> this CTA's shared memory, completing `bytes` on `bar`.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),

@@ -500,7 +500,11 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
                   make_float2(fos[v / BT][v % BT], fos[(v + 1) / BT][(v + 1) % BT]);
           } else {
             st_async_v2f64(ra_ + 8u * v, o0, o1, rbar);
-            if constexpr (ADJ) st_async_v2f32(rf_ + 4u * v, fos[v / BT][v % BT], fos[(v + 1) / BT][(v + 1) % BT], rbar);
+            if constexpr (ADJ) {  // four accumulators per store (U * BT is 4 or 8)
+              if (v % 4 == 0)
+                st_async_v4f32(rf_ + 4u * v, fos[v / BT][v % BT], fos[(v + 1) / BT][(v + 1) % BT],
+                               fos[(v + 2) / BT][(v + 2) % BT], fos[(v + 3) / BT][(v + 3) % BT], rbar);
+            }
           }
         }
       } else {
@@ -771,6 +775,12 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
                         ? p.marginals + (static_cast<size_t>(c.seq) * n + t) * static_cast<size_t>(S)
                         : nullptr;
       const bool send = t >= 1;
+      // K = 4 cluster teams of the adjoint send the float32 accumulators of two
+      // neighbouring groups (adjacent slots of one CTA) per store: the two
+      // lanes of a pair swap their values of row jj and one of them stores
+      // both.  (Measured: this halves the cost of the accumulators' exchange;
+      // pairing the float64 outputs the same way costs more than it saves.)
+      constexpr bool kPairBt = CL > 1 && K == 4 && ADJ;
       // The state loop, instantiated with and without the marginal stores so
       // that a call without marginals carries none of their addressing.
       auto states = [&](auto with_marginals) {
@@ -831,7 +841,16 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
             } else {
               const uint32_t rbar = mapa_u32(bar_l, rk);
               st_async_f64(mapa_u32(smem_u32(exB_w + off), rk), out, rbar);
-              if constexpr (ADJ) st_async_f32(mapa_u32(smem_u32(exBt_w + off), rk), bt_out, rbar);
+              if constexpr (kPairBt) {
+                // lanes 2i and 2i + 1 hold groups q0 - odd and q0 - odd + 1
+                const int odd = tm.lane & 1;
+                const float f_pair = __shfl_xor_sync(fbk::kFull, bt_out, 1);
+                if (odd == (jj & 1))
+                  st_async_v2f32(mapa_u32(smem_u32(exBt_w + off - odd), rk), odd ? f_pair : bt_out,
+                                 odd ? bt_out : f_pair, rbar);
+              } else if constexpr (ADJ) {
+                st_async_f32(mapa_u32(smem_u32(exBt_w + off), rk), bt_out, rbar);
+              }
             }
           }
         }

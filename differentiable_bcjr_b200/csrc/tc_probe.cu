@@ -111,6 +111,61 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kXThreads, 1)
   cluster_sync_all();  // no CTA leaves while its shared memory may be addressed
 }
 
+constexpr uint32_t kXSmemBulk = 4 * kXSlot + 64;  // three receive slots, one source slot, the mbarrier
+
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t rbar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   dst),
+               "r"(src), "r"(bytes), "r"(rbar)
+               : "memory");
+}
+
+// The same exchange as dsmem_probe_kernel, moved by the bulk-copy engine: each
+// warp owns 4 KiB of every 32 KiB slot and its lanes issue one
+// cp.async.bulk (shared::cta -> shared::cluster, completing on the receiver's
+// mbarrier) per `chunk` bytes of it, from a local source slot written once.
+__global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kXThreads, 1)
+    dsmem_bulk_probe_kernel(int chunk, int reps, int rounds, long long* __restrict__ cycles, int* __restrict__ status) {
+  extern __shared__ __align__(1024) unsigned char sm[];
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + 4 * kXSlot);
+  float4* src = reinterpret_cast<float4*>(sm + 3 * kXSlot);
+  const uint32_t rank = cluster_rank();
+  for (int i = threadIdx.x; i < static_cast<int>(kXSlot / 16); i += kXThreads)
+    src[i] = make_float4(1.f, 2.f, 3.f, static_cast<float>(i));
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    mbar_init_fence();
+  }
+  async_proxy_fence();  // the source's generic-proxy writes before the copies read it
+  __syncthreads();
+  cluster_sync_all();
+  constexpr uint32_t kPerWarp = kXSlot / (kXThreads / 32);
+  const uint32_t ch = static_cast<uint32_t>(chunk);
+  const uint32_t nch = kPerWarp / ch;
+  const uint32_t warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t total = 3u * kXSlot * static_cast<uint32_t>(reps);
+  const uint32_t src_base = smem_u32(src) + warp * kPerWarp;
+  bool timed_out = false;
+  const long long t0 = clock64();
+  for (int it = 0; it < rounds; ++it) {
+    if (threadIdx.x == 0) mbar_arm(bar, total);
+    cluster_arrive_relaxed();
+    cluster_wait_plain();
+    for (int rep = 0; rep < reps; ++rep)
+      for (uint32_t i = lane; i < 3u * nch; i += 32u) {
+        const uint32_t peer = (rank + 1u + i / nch) & 3u;
+        const uint32_t c = i % nch;
+        const uint32_t sl = rank < peer ? rank : rank - 1;
+        const uint32_t dst = mapa_u32(smem_u32(sm) + sl * kXSlot + warp * kPerWarp + c * ch, peer);
+        bulk_copy_to_peer(dst, src_base + c * ch, ch, mapa_u32(smem_u32(bar), peer));
+      }
+    if (!timed_out) timed_out = !mbar_wait(bar, static_cast<uint32_t>(it & 1), status, kDevTimeout);
+  }
+  const long long t1 = clock64();
+  if (threadIdx.x == 0) cycles[blockIdx.x] = t1 - t0;
+  cluster_sync_all();
+}
+
 }  // namespace
 
 extern "C" bcjr_status bcjr_probe_mma_tf32(int n, int iters, long long* cycles, int* status, int n_sm,
@@ -146,6 +201,22 @@ extern "C" bcjr_status bcjr_probe_dsmem(int reps, int rounds, long long* cycles,
   if (e == cudaSuccess) {
     dsmem_probe_kernel<<<4 * n_clusters, kXThreads, kXSmem, reinterpret_cast<cudaStream_t>(stream)>>>(
         reps, rounds, cycles, status);
+    e = cudaGetLastError();
+  }
+  return e == cudaSuccess ? BCJR_OK : BCJR_ERR_CUDA;
+}
+
+extern "C" bcjr_status bcjr_probe_dsmem_bulk(int chunk_bytes, int reps, int rounds, long long* cycles, int* status,
+                                             int n_clusters, bcjr_stream_t stream) {
+  const bool chunk_ok = chunk_bytes >= 128 && chunk_bytes <= 4096 && (chunk_bytes & (chunk_bytes - 1)) == 0;
+  if (!chunk_ok || reps < 1 || reps > 8 || rounds < 1 || rounds > (1 << 16) || !cycles || !status ||
+      n_clusters < 1 || n_clusters > 1024)
+    return BCJR_ERR_INVALID_ARG;
+  cudaError_t e =
+      cudaFuncSetAttribute(dsmem_bulk_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kXSmemBulk);
+  if (e == cudaSuccess) {
+    dsmem_bulk_probe_kernel<<<4 * n_clusters, kXThreads, kXSmemBulk, reinterpret_cast<cudaStream_t>(stream)>>>(
+        chunk_bytes, reps, rounds, cycles, status);
     e = cudaGetLastError();
   }
   return e == cudaSuccess ? BCJR_OK : BCJR_ERR_CUDA;

@@ -68,13 +68,21 @@ bcjr_status bcjr_probe_xu(int op, int iters, float* sink, long long* cycles, int
  *   status      as above
  *   n_clusters  clusters launched, 1 .. 1024 (clusters beyond those that fit
  *               at once run later and measure the same)
- * Both are asynchronous on `stream`; they return BCJR_ERR_INVALID_ARG for bad
- * sizes or null pointers and BCJR_ERR_CUDA if the launch fails.
+ * bcjr_probe_dsmem_bulk: the same exchange (sizes, rounds, cycles) moved by
+ * the bulk-copy engine instead of per-thread stores: every warp owns 4 KiB of
+ * each 32 KiB slot and issues one cp.async.bulk from a local shared-memory
+ * source into the peer's slot per `chunk_bytes` (a power of two, 128 .. 4096),
+ * completing on the receiver's mbarrier.
+ *
+ * All three are asynchronous on `stream`; they return BCJR_ERR_INVALID_ARG for
+ * bad sizes or null pointers and BCJR_ERR_CUDA if the launch fails.
  */
 bcjr_status bcjr_probe_mma_tf32(int n, int iters, long long* cycles, int* status, int n_sm,
                                 bcjr_stream_t stream);
 bcjr_status bcjr_probe_dsmem(int reps, int rounds, long long* cycles, int* status, int n_clusters,
                              bcjr_stream_t stream);
+bcjr_status bcjr_probe_dsmem_bulk(int chunk_bytes, int reps, int rounds, long long* cycles, int* status,
+                                  int n_clusters, bcjr_stream_t stream);
 
 #ifdef __cplusplus
 }

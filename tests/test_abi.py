@@ -31,7 +31,8 @@ def test_header_declares_the_calls():
     for required in ["bcjr_forward", "bcjr_backward", "viterbi_decode", "bcjr_workspace_size",
                      "bcjr_get_status", "bcjr_status_string", "bcjr_dense_forward", "bcjr_dense_backward",
                      "bcjr_dense_backward_lambda", "bcjr_forward_static_scratch", "bcjr_static_scratch_status",
-                     "bcjr_probe_xu", "bcjr_probe_mma_tf32", "bcjr_probe_dsmem"]:
+                     "bcjr_probe_xu", "bcjr_probe_mma_tf32", "bcjr_probe_dsmem",
+                     "bcjr_probe_dsmem_bulk"]:
         assert required in names, names
 
 

@@ -28,6 +28,7 @@ def test_mma_probe(B, n):
     assert 4 < r["clk_per_mma"] < 2000
 
 
-def test_dsmem_probe(B):
-    r = B.probe_dsmem(2, 20)
+@pytest.mark.parametrize("chunk", [0, 256, 4096])
+def test_dsmem_probe(B, chunk):
+    r = B.probe_dsmem(2, 20, chunk=chunk)
     assert 1.0 < r["bytes_per_clk_per_sm"] < 256.0
