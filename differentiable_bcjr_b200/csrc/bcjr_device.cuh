@@ -279,6 +279,20 @@ __device__ __forceinline__ void st_async_v4f32(uint32_t raddr, float a, float b,
                "f"(a), "f"(b), "f"(c), "f"(d), "r"(rbar)
                : "memory");
 }
+// Bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned) from
+// this CTA's shared memory at `src` into cluster shared memory at `dst`,
+// completing on the mbarrier at `rbar` (dst and rbar mapped to the destination
+// CTA).  The source must stay unchanged until the destination's mbarrier
+// phase has completed.
+__device__ __forceinline__ void bulk_copy_s2c(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t rbar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   dst),
+               "r"(src), "r"(bytes), "r"(rbar)
+               : "memory");
+}
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy operations (bulk copies, tensor-core reads) on them.
+__device__ __forceinline__ void async_proxy_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 // Split cluster barrier without memory ordering: it only orders the
 // execution of the threads (every read of a buffer before its next overwrite).
 __device__ __forceinline__ void cluster_arrive_relaxed() {

@@ -241,7 +241,11 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
   constexpr double kRefOff = static_cast<double>(k + 1) * fbk::kScale;
 
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  const FBSmem lay = fb_smem_layout(GL, NT, NV, NSEQ, ADJ, alias, tpc);
+  // Forward-call cluster teams (K <= 4, up to two sequences in flight) stage a
+  // warp's outgoing forward-sweep values in their own shared memory and send
+  // them as one bulk copy: one copy per warp instead of a store per thread.
+  constexpr bool kBulk = CL > 1 && !ADJ && K <= 4 && NSEQ <= 2;
+  const FBSmem lay = fb_smem_layout(GL, NT, NV, NSEQ, ADJ, alias, tpc, kBulk);
   unsigned char* team_base = smem_raw + static_cast<size_t>(team_in_cta) * lay.per_team;
   float* red = reinterpret_cast<float*>(smem_raw + lay.red);
   float* redk = reinterpret_cast<float*>(smem_raw + lay.red) + 256;
@@ -489,6 +493,22 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
           rbar = mapa_u32(bar_l, r);
           ra_ = mapa_u32(smem_u32(exA_w + off), r);
           if constexpr (ADJ) rf_ = mapa_u32(smem_u32(exF_w + off), r);
+        }
+        if constexpr (kBulk) {
+          // The warp's 32 x U*BT values are consecutive slots of one CTA: stage
+          // them in the same order (slot parity and sequence of their own) and
+          // let lane 0 copy the block.  The staging slot is rewritten two steps
+          // later, after the barrier that follows every reader's wait for it.
+          double* stg = reinterpret_cast<double*>(smem_raw + lay.xst) + (X * 2 + ((t + 1) & 1)) * GL;
+#pragma unroll
+          for (int v = 0; v < U * BT; v += 2)
+            *reinterpret_cast<double2*>(stg + threadIdx.x * (U * BT) + v) =
+                make_double2(outs[v / BT][v % BT], outs[(v + 1) / BT][(v + 1) % BT]);
+          async_proxy_fence();
+          __syncwarp();
+          if (tm.lane == 0)
+            bulk_copy_s2c(ra_, smem_u32(stg + threadIdx.x * (U * BT)), 32u * U * BT * 8u, rbar);
+          return;
         }
 #pragma unroll
         for (int v = 0; v < U * BT; v += 2) {

@@ -113,13 +113,6 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kXThreads, 1)
 
 constexpr uint32_t kXSmemBulk = 4 * kXSlot + 64;  // three receive slots, one source slot, the mbarrier
 
-__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t rbar) {
-  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   dst),
-               "r"(src), "r"(bytes), "r"(rbar)
-               : "memory");
-}
-
 // The same exchange as dsmem_probe_kernel, moved by the bulk-copy engine: each
 // warp owns 4 KiB of every 32 KiB slot and its lanes issue one
 // cp.async.bulk (shared::cta -> shared::cluster, completing on the receiver's
@@ -157,7 +150,7 @@ __global__ void __cluster_dims__(4, 1, 1) __launch_bounds__(kXThreads, 1)
         const uint32_t c = i % nch;
         const uint32_t sl = rank < peer ? rank : rank - 1;
         const uint32_t dst = mapa_u32(smem_u32(sm) + sl * kXSlot + warp * kPerWarp + c * ch, peer);
-        bulk_copy_to_peer(dst, src_base + c * ch, ch, mapa_u32(smem_u32(bar), peer));
+        bulk_copy_s2c(dst, src_base + c * ch, ch, mapa_u32(smem_u32(bar), peer));
       }
     if (!timed_out) timed_out = !mbar_wait(bar, static_cast<uint32_t>(it & 1), status, kDevTimeout);
   }
