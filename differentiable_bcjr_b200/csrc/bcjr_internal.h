@@ -64,10 +64,12 @@ struct FBParams {
 // values read by the backward sweep (values, reference words, accumulators),
 // and every thread's float codewords.
 struct FBSmem {
-  uint32_t exA, exF, exB, exBt, mbar, per_seq, per_team, red, stage, stageK, stageF, xst, cf, total;
+  uint32_t exA, exF, exB, exBt, mbar, per_seq, per_team, red, stage, stageK, stageF, xst, xstF, cf, total;
 };
-// `xstage`: the outgoing forward-sweep group values are staged here per
-// sequence in flight and parity (GL float64 each) and leave by bulk copy.
+// `xstage`: outgoing group values are staged per sequence in flight and
+// parity (GL float64, and GL float32 accumulators for the adjoint) and leave
+// by bulk copy.  The adjoint stages its forward sweep only, so its staging
+// shares room with the checkpoint staging, which only its backward sweep uses.
 __host__ __device__ inline FBSmem fb_smem_layout(int GL, int NT, int NV, int nseq, bool adj, bool alias,
                                                  int teams_per_cta, bool xstage) {
   FBSmem l;
@@ -97,8 +99,10 @@ __host__ __device__ inline FBSmem fb_smem_layout(int GL, int NT, int NV, int nse
   l.stageK = o;
   o += stg * 4u;
   o = (o + 15u) & ~15u;
-  l.xst = o;
-  if (xstage) o += static_cast<uint32_t>(nseq) * 2u * GL * 8u;
+  l.xst = adj ? l.stage : o;
+  l.xstF = l.xst + static_cast<uint32_t>(nseq) * 2u * GL * 8u;
+  const uint32_t xend = l.xstF + (adj ? static_cast<uint32_t>(nseq) * 2u * GL * 4u : 0u);
+  if (xstage && xend > o) o = (xend + 15u) & ~15u;
   l.cf = o;  // float codewords of every thread: [8 pairs][NT] float2
   o += static_cast<uint32_t>(NT) * 16u * 4u;
   l.total = o;

@@ -241,11 +241,16 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
   constexpr double kRefOff = static_cast<double>(k + 1) * fbk::kScale;
 
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  // Forward-call cluster teams (K <= 4, up to two sequences in flight) stage a
-  // warp's outgoing forward-sweep values in their own shared memory and send
-  // them as one bulk copy: one copy per warp instead of a store per thread.
-  constexpr bool kBulk = CL > 1 && !ADJ && K <= 4 && NSEQ <= 2;
-  const FBSmem lay = fb_smem_layout(GL, NT, NV, NSEQ, ADJ, alias, tpc, kBulk);
+  // In the forward sweep, cluster teams with K <= 4 and up to two sequences in
+  // flight stage a warp's outgoing values in their own shared memory and send
+  // them as one bulk copy instead of a store per thread (the adjoint only with
+  // C = 1: with C > 1 its backward buffers leave no room).  The backward
+  // sweep keeps per-thread stores: a warp's outputs there form one block per
+  // output row, and four staged copies per step measured slower than the
+  // stores.
+  constexpr bool kBulk = CL > 1 && K <= 4 && NSEQ <= 2;
+  const bool xst_on = kBulk && (!ADJ || alias);
+  const FBSmem lay = fb_smem_layout(GL, NT, NV, NSEQ, ADJ, alias, tpc, xst_on);
   unsigned char* team_base = smem_raw + static_cast<size_t>(team_in_cta) * lay.per_team;
   float* red = reinterpret_cast<float*>(smem_raw + lay.red);
   float* redk = reinterpret_cast<float*>(smem_raw + lay.red) + 256;
@@ -494,20 +499,30 @@ __global__ void __launch_bounds__(NTB, 1) fb_kernel(const FBParams p) {
           ra_ = mapa_u32(smem_u32(exA_w + off), r);
           if constexpr (ADJ) rf_ = mapa_u32(smem_u32(exF_w + off), r);
         }
-        if constexpr (kBulk) {
+        if (xst_on) {
           // The warp's 32 x U*BT values are consecutive slots of one CTA: stage
           // them in the same order (slot parity and sequence of their own) and
           // let lane 0 copy the block.  The staging slot is rewritten two steps
           // later, after the barrier that follows every reader's wait for it.
-          double* stg = reinterpret_cast<double*>(smem_raw + lay.xst) + (X * 2 + ((t + 1) & 1)) * GL;
+          const int sidx = (X * 2 + ((t + 1) & 1)) * GL + threadIdx.x * (U * BT);
+          double* stg = reinterpret_cast<double*>(smem_raw + lay.xst) + sidx;
+          float* stgF = reinterpret_cast<float*>(smem_raw + lay.xstF) + sidx;
 #pragma unroll
           for (int v = 0; v < U * BT; v += 2)
-            *reinterpret_cast<double2*>(stg + threadIdx.x * (U * BT) + v) =
-                make_double2(outs[v / BT][v % BT], outs[(v + 1) / BT][(v + 1) % BT]);
+            *reinterpret_cast<double2*>(stg + v) = make_double2(outs[v / BT][v % BT], outs[(v + 1) / BT][(v + 1) % BT]);
+          if constexpr (ADJ) {
+#pragma unroll
+            for (int v = 0; v < U * BT; v += 4)
+              *reinterpret_cast<float4*>(stgF + v) =
+                  make_float4(fos[v / BT][v % BT], fos[(v + 1) / BT][(v + 1) % BT], fos[(v + 2) / BT][(v + 2) % BT],
+                              fos[(v + 3) / BT][(v + 3) % BT]);
+          }
           async_proxy_fence();
           __syncwarp();
-          if (tm.lane == 0)
-            bulk_copy_s2c(ra_, smem_u32(stg + threadIdx.x * (U * BT)), 32u * U * BT * 8u, rbar);
+          if (tm.lane == 0) {
+            bulk_copy_s2c(ra_, smem_u32(stg), 32u * U * BT * 8u, rbar);
+            if constexpr (ADJ) bulk_copy_s2c(rf_, smem_u32(stgF), 32u * U * BT * 4u, rbar);
+          }
           return;
         }
 #pragma unroll
