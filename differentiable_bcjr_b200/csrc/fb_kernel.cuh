@@ -47,6 +47,13 @@
 //  * The exchange buffers a sweep starts from are zero-filled (A_0 = 0,
 //    B_{n-1} = 0), so every step reads them without a select.
 //
+// Exchange.  On a cluster, group values go straight into the shared memory of
+// the CTA that reads them next step, completing on that CTA's mbarrier.  In
+// the forward sweep a warp's outputs are one block of consecutive slots: they
+// are staged in the sending CTA and leave as one bulk copy per warp.  In the
+// backward sweep each thread's outputs go to four CTAs and leave as
+// per-thread st.async stores.
+//
 // Schedule.  A team (thread-block cluster, one CTA, or a slice of a warp)
 // keeps NSEQ sequences in flight.  With NSEQ = 2 the steps of the two
 // sequences alternate and each step ends with a split cluster barrier whose
@@ -135,9 +142,10 @@ __device__ __forceinline__ float2 group_sum2(float2 v, int width) {
 // Barrier schedule of one team.  With NSEQ >= 2 on a cluster: after block b,
 // wait for the phase of block b-1 (the previous sequence's block) and arrive
 // for block b.  Global stores go after the arrive.
-// On a cluster the exchanged data travel with st.async and are awaited on
-// mbarriers, so this barrier orders execution only (every read of a buffer
-// before its overwrite two steps later) and carries no memory fence.
+// On a cluster the exchanged data travel with st.async or bulk copies and are
+// awaited on mbarriers, so this barrier orders execution only (every read of a
+// buffer, and every bulk copy's read of its staging block, before the
+// overwrite two steps later) and carries no memory fence.
 template <int CL, int NSEQ>
 struct Pipe {
   bool pending = false;
