@@ -57,6 +57,13 @@ struct FBParams {
   long long probe_wait_cycles;  // > 0: only the bounded-wait probe runs (testing aid)
 };
 
+// Whether a forward-backward launch stages its outgoing forward-sweep values
+// for bulk copies (fb_kernel's xst_on): cluster teams with k <= 2 and up to
+// two sequences in flight; the adjoint only with C = 1 (`alias`).
+__host__ __device__ inline bool fb_xstage(int cluster, int k, int nseq, bool adj, bool alias) {
+  return cluster > 1 && k <= 2 && nseq <= 2 && (!adj || alias);
+}
+
 // Shared-memory carve-up of the forward-backward kernel (bytes), identical on
 // host and device.  Per team and per sequence in flight: the double-buffered
 // exchange vectors (float64 group values, float32 adjoint accumulators); per

@@ -204,7 +204,7 @@ cudaError_t fb_geometry_uncached(int L, int k, int n_seq, bool adjoint, int C, i
       return cudaErrorNotSupported;
     nseq = nseq_request;
   }
-  const bool xstage = g->cluster > 1 && k <= 2 && nseq <= 2 && (!adjoint || alias);  // as xst_on in fb_kernel
+  const bool xstage = fb_xstage(g->cluster, k, nseq, adjoint, alias);
   const size_t smem =
       fb_smem_layout(GL, g->block_threads, NV, nseq, adjoint, alias, g->teams_per_cta, xstage).total;
   if (smem > static_cast<size_t>(max_smem)) return cudaErrorNotSupported;
