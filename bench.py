@@ -453,8 +453,9 @@ def run_mufu(args):
 
 def run_tcprobe(args):
     """The two costs that bound a step of the dense tensor-core kernels: the
-    issue cost of a tf32 tensor-core product by N, and the st.async exchange
-    bandwidth between the CTAs of 4-CTA clusters (all SMs, and a few)."""
+    issue cost of a tf32 tensor-core product by N, and the exchange bandwidth
+    between the CTAs of 4-CTA clusters (st.async on all SMs and on a few; bulk
+    copies of 256 B, 1 KiB and 4 KiB on all SMs)."""
     world, rank, local = dist_env()
     if rank != 0:
         return 0
@@ -472,6 +473,10 @@ def run_tcprobe(args):
     xfew = [B.probe_dsmem(reps, rounds, 2, dev) for _ in range(steps)]
     bw_all = statistics.median(x["bytes_per_clk_per_sm"] for x in xall)
     bw_few = statistics.median(x["bytes_per_clk_per_sm"] for x in xfew)
+    # the same exchange moved by bulk copies of `chunk` bytes (every SM)
+    chunks = (256, 1024, 4096)
+    bulk = {c: statistics.median(B.probe_dsmem(reps, rounds, 0, dev, chunk=c)["bytes_per_clk_per_sm"]
+                                 for _ in range(steps)) for c in chunks}
     line = {"metric": "tcgen05 tf32 product issue cost (M=128, K=8, A in tensor memory) and 4-CTA-cluster "
                       "st.async exchange bandwidth",
             "value": bw_all, "unit": "bytes/clk/SM", "n_gpus": 1, "steps": steps, "warmup": args.warmup,
@@ -481,7 +486,8 @@ def run_tcprobe(args):
             "mma_clk_per_product": {str(n): c for n, c in mma.items()},
             "mma_mac_per_clk_per_sm": {str(n): 128.0 * n * 8 / c for n, c in mma.items()},
             "dsmem_bytes_per_clk_per_sm": {"all_sms": bw_all, "two_clusters": bw_few},
-            "gpu_launches": 5 * steps + 2 * steps + 2 * max(args.warmup, 1)}
+            "dsmem_bulk_bytes_per_clk_per_sm": {str(c): v for c, v in bulk.items()},
+            "gpu_launches": 5 * steps + 2 * steps + len(chunks) * steps + 2 * max(args.warmup, 1)}
     print(json.dumps(line), flush=True)
     return 0
 
