@@ -1,9 +1,10 @@
 // tc_probe.cu -- measurement aids behind the dense trellis's tensor-core
-// design: the issue cost of one tf32 tensor-core product (tcgen05.mma with
-// operand A in tensor memory) as a function of N, and the bandwidth of the
-// distributed-shared-memory exchange between the CTAs of a 4-CTA cluster.
-// They are what bound a step of the dense kernels (the per-step reduce-scatter
-// and the per-step MMAs), measured on the device at hand.
+// design and the clusters' exchange: the issue cost of one tf32 tensor-core
+// product (tcgen05.mma with operand A in tensor memory) as a function of N,
+// and the bandwidth of the distributed-shared-memory exchange between the
+// CTAs of a 4-CTA cluster, moved by per-thread st.async stores or by bulk
+// copies.  They are what bound a step of the dense kernels (the per-step
+// reduce-scatter and the per-step MMAs), measured on the device at hand.
 #include <cuda_runtime.h>
 
 #include <cstdint>
